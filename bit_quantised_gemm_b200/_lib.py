@@ -1,0 +1,262 @@
+"""ctypes binding of libbitlinear.so: argument marshalling only.
+
+Every computation happens in the CUDA library; this module passes device
+pointers, sizes and the current CUDA stream, allocates outputs with torch,
+and turns error codes into exceptions. There is no CPU fallback: if the
+library is missing, every call raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libbitlinear.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "bitlinear.h")
+
+MODE_INT8, MODE_INT4, MODE_FP4 = 0, 1, 2
+OK, ERR_INVALID_ARG, ERR_ALIGNMENT, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+STATUS_TIMEOUT = 1
+
+
+class BitlinearError(RuntimeError):
+    def __init__(self, code: int, msg: str):
+        super().__init__(f"bitlinear error {code}: {msg}")
+        self.code = code
+
+
+_c = ctypes
+_P = _c.c_void_p
+_I64 = _c.c_int64
+_INT = _c.c_int
+
+_SIGS = {
+    "bitlinear_last_error": ([], _c.c_char_p),
+    "bitlinear_version": ([], _INT),
+    "bitlinear_set_wait_timeout_ns": ([_I64], _INT),
+    "bitlinear_ternarize_pack": ([_P, _I64, _I64, _P, _INT, _P, _P], _INT),
+    "bitlinear_quant_act": ([_P, _P, _I64, _I64, _I64, _INT, _P, _P, _P], _INT),
+    "bitlinear_topk_sparsify_i8": ([_P, _I64, _I64, _I64, _I64, _P, _P, _P, _P], _INT),
+    "bitlinear_gemm_w2a8": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
+    "bitlinear_gemm_w2a4": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
+    "bitlinear_gemm_w2fp4": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
+    "bitlinear_gemm_w2a8_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
+    "bitlinear_gemm_w2fp4_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
+    "bitlinear_gemv_w2": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
+    "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
+    "bitlinear_check_status": ([_P, _P], _INT),
+    "bitlinear_debug_wait_timeout": ([_P, _I64, _P], _INT),
+}
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libbitlinear.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m bit_quantised_gemm_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (args, res) in _SIGS.items():
+            f = getattr(L, name)
+            f.argtypes = args
+            f.restype = res
+        _lib = L
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions declared in include/bitlinear.h."""
+    text = open(HEADER_PATH).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def _check(rc: int):
+    if rc != OK:
+        raise BitlinearError(rc, lib().bitlinear_last_error().decode())
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    return t.data_ptr()
+
+
+def _stream(stream=None) -> int:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def _require_cuda(*ts):
+    for t in ts:
+        if t is not None and not t.is_cuda:
+            raise ValueError("expected a CUDA tensor")
+
+
+def _rows(t: torch.Tensor) -> tuple[int, int, int]:
+    """(M, K, ld) of a 2-D tensor whose rows are contiguous."""
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D tensor with contiguous rows")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+_status = {}
+
+
+def status_buffer(device=None) -> torch.Tensor:
+    """Per-device int32 status word passed to the GEMM kernels (zeroed)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    if key not in _status:
+        _status[key] = torch.zeros(1, dtype=torch.int32, device=f"cuda:{key}")
+    return _status[key]
+
+
+# ------------------------------------------------------------------ API
+def version() -> int:
+    return lib().bitlinear_version()
+
+
+def set_wait_timeout_ns(ns: int):
+    _check(lib().bitlinear_set_wait_timeout_ns(int(ns)))
+
+
+def ternarize_pack(W: np.ndarray, group_ends) -> tuple[np.ndarray, np.ndarray]:
+    """Host weight prep: fp32 W [K x N] -> (Wp uint8 [N x K/4], gamma fp32 [G])."""
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    K, N = W.shape
+    ge = np.ascontiguousarray(group_ends, dtype=np.int64)
+    Wp = np.zeros((N, K // 4), dtype=np.uint8)
+    gamma = np.zeros(len(ge), dtype=np.float32)
+    _check(lib().bitlinear_ternarize_pack(_ptr(W), K, N, _ptr(ge), len(ge), _ptr(Wp), _ptr(gamma)))
+    return Wp, gamma
+
+
+def quant_act(x: torch.Tensor, mode: int, up: torch.Tensor | None = None, out=None, xs=None,
+              stream=None):
+    """Per-token quantiser (INT8 / INT4 / FP4), optionally of relu(x)^2 * up."""
+    _require_cuda(x, up)
+    M, K, ld = _rows(x)
+    if up is not None and (up.shape != x.shape or up.stride() != x.stride()):
+        raise ValueError("up must match x in shape and strides")
+    if out is None:
+        out = (torch.empty((M, K // 2), dtype=torch.uint8, device=x.device) if mode == MODE_FP4
+               else torch.empty((M, K), dtype=torch.int8, device=x.device))
+    if xs is None:
+        xs = torch.empty(M, dtype=torch.float32, device=x.device)
+    _check(lib().bitlinear_quant_act(_ptr(x), _ptr(up), M, K, ld, mode, _ptr(out), _ptr(xs),
+                                     _stream(stream)))
+    return out, xs
+
+
+def topk_sparsify_i8(x: torch.Tensor, k: int = 0, mask: bool = False, out=None, xs=None,
+                     stream=None):
+    """Keep the k (default ceil(K/2)) largest |x| per row, zero the rest, INT8."""
+    _require_cuda(x)
+    M, K, ld = _rows(x)
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.int8, device=x.device)
+    if xs is None:
+        xs = torch.empty(M, dtype=torch.float32, device=x.device)
+    mk = torch.empty((M, K // 8), dtype=torch.uint8, device=x.device) if mask else None
+    _check(lib().bitlinear_topk_sparsify_i8(_ptr(x), M, K, ld, int(k), _ptr(out), _ptr(xs),
+                                            _ptr(mk), _stream(stream)))
+    return out, xs, mk
+
+
+def _gemm(fn: str, a: torch.Tensor, xs, Wp, gamma, group_ends, K: int, y=None, status=None,
+          stream=None):
+    _require_cuda(a, xs, Wp, gamma)
+    M = a.shape[0]
+    N = Wp.shape[0]
+    ge = np.ascontiguousarray(group_ends, dtype=np.int64)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    if status is None:
+        status = status_buffer(a.device)
+    _check(getattr(lib(), fn)(_ptr(a), _ptr(xs), _ptr(Wp), _ptr(gamma), _ptr(ge), len(ge), M, N, K,
+                              _ptr(y), y.stride(0), _ptr(status), _stream(stream)))
+    return y
+
+
+def gemm_w2a8(xq, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
+    """y = bf16((xq @ W_t) * xs[m] * gamma[group(n)]) on tensor cores (int8 codes)."""
+    return _gemm("bitlinear_gemm_w2a8", xq, xs, Wp, gamma, group_ends, xq.shape[1], y, status, stream)
+
+
+def gemm_w2a4(xq, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
+    """As gemm_w2a8 for INT4 codes held in int8."""
+    return _gemm("bitlinear_gemm_w2a4", xq, xs, Wp, gamma, group_ends, xq.shape[1], y, status, stream)
+
+
+def gemm_w2fp4(xf4, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
+    """As gemm_w2a8 for packed e2m1 activations [M x K/2]."""
+    return _gemm("bitlinear_gemm_w2fp4", xf4, xs, Wp, gamma, group_ends, 2 * xf4.shape[1], y,
+                 status, stream)
+
+
+def gemv_w2(xq, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
+    """Decode-time variant of gemm_w2a8 for 1..64 tokens."""
+    return _gemm("bitlinear_gemv_w2", xq, xs, Wp, gamma, group_ends, xq.shape[1], y, status, stream)
+
+
+def gemm_w2a8_acc(xq, Wp, status=None, stream=None):
+    """Raw int32 accumulators [M x N] of the int8 GEMM."""
+    _require_cuda(xq, Wp)
+    M, K = xq.shape
+    N = Wp.shape[0]
+    acc = torch.empty((M, N), dtype=torch.int32, device=xq.device)
+    status = status if status is not None else status_buffer(xq.device)
+    _check(lib().bitlinear_gemm_w2a8_acc(_ptr(xq), _ptr(Wp), M, N, K, _ptr(acc), _ptr(status),
+                                         _stream(stream)))
+    return acc
+
+
+def gemm_w2fp4_acc(xf4, Wp, status=None, stream=None):
+    """Raw fp32 accumulators [M x N] of the FP4 GEMM."""
+    _require_cuda(xf4, Wp)
+    M, Kh = xf4.shape
+    N = Wp.shape[0]
+    acc = torch.empty((M, N), dtype=torch.float32, device=xf4.device)
+    status = status if status is not None else status_buffer(xf4.device)
+    _check(lib().bitlinear_gemm_w2fp4_acc(_ptr(xf4), _ptr(Wp), M, N, 2 * Kh, _ptr(acc),
+                                          _ptr(status), _stream(stream)))
+    return acc
+
+
+def kv_quant_3bit(kv: torch.Tensor, keep4_pos: torch.Tensor | None, codes3=None, codes4=None,
+                  scale=None, stream=None):
+    """3-bit per-(token, head) KV quantiser; listed tokens at 4 bits."""
+    _require_cuda(kv, keep4_pos)
+    if kv.dim() != 3 or not kv.is_contiguous():
+        raise ValueError("kv must be a contiguous [T x H x D] tensor")
+    T, H, D = kv.shape
+    n4 = 0 if keep4_pos is None else keep4_pos.numel()
+    if codes3 is None:
+        codes3 = torch.empty((T, H, 3 * D // 8), dtype=torch.uint8, device=kv.device)
+    if codes4 is None and n4:
+        codes4 = torch.empty((n4, H, D // 2), dtype=torch.uint8, device=kv.device)
+    if scale is None:
+        scale = torch.empty((T, H), dtype=torch.float32, device=kv.device)
+    _check(lib().kv_quant_3bit(_ptr(kv), T, H, D, _ptr(keep4_pos), n4, _ptr(codes3), _ptr(codes4),
+                               _ptr(scale), _stream(stream)))
+    return codes3, codes4, scale
+
+
+def check_status(status: torch.Tensor | None = None, stream=None):
+    """Synchronise and raise BitlinearError(ERR_TIMEOUT) if a kernel gave up a wait."""
+    status = status if status is not None else status_buffer()
+    _check(lib().bitlinear_check_status(_ptr(status), _stream(stream)))
+
+
+def debug_wait_timeout(status: torch.Tensor, timeout_ns: int, stream=None):
+    _check(lib().bitlinear_debug_wait_timeout(_ptr(status), int(timeout_ns), _stream(stream)))

@@ -1,0 +1,72 @@
+// Shared definitions for the BitLinear kernels: launch parameters, the
+// ternary-weight unpack, and small numeric helpers.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cstdint>
+
+namespace blt {
+
+constexpr float kEps = 1e-5f;  // floor of every absmax scale
+
+// ----------------------------------------------------------- bf16 helpers
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+  f[0] = bf16lo(v.x); f[1] = bf16hi(v.x);
+  f[2] = bf16lo(v.y); f[3] = bf16hi(v.y);
+  f[4] = bf16lo(v.z); f[5] = bf16hi(v.z);
+  f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// ------------------------------------------------------ ternary unpacking
+// A 32-bit word of the packed weights holds 16 consecutive k: element 8h+i
+// sits in bits [4i+2h, 4i+2h+2) as code c = w + 1 (0, 1, 2). Masking with
+// 0x33333333 after a shift of 2h leaves one code per nibble, which PRMT
+// then uses as a byte selector into a 4-entry lookup table.
+__device__ __forceinline__ uint32_t codes_lo(uint32_t w) { return w & 0x33333333u; }
+__device__ __forceinline__ uint32_t codes_hi(uint32_t w) { return (w >> 2) & 0x33333333u; }
+
+// 16 weights -> 16 signed int8 bytes in k order (-1 -> 0xFF, 0, +1 -> 0x01).
+__device__ __forceinline__ uint4 unpack16_s8(uint32_t w) {
+  constexpr uint32_t kLut = 0x000100FFu;  // code 0 -> -1, 1 -> 0, 2 -> +1, 3 -> 0
+  const uint32_t x0 = codes_lo(w), x1 = codes_hi(w);
+  uint4 o;
+  o.x = __byte_perm(kLut, 0u, x0);
+  o.y = __byte_perm(kLut, 0u, x0 >> 16);
+  o.z = __byte_perm(kLut, 0u, x1);
+  o.w = __byte_perm(kLut, 0u, x1 >> 16);
+  return o;
+}
+
+// One nibble per code -> e2m1 nibble: code 0 -> 0xA (-1.0), 1 -> 0x0, 2 -> 0x2 (+1.0).
+__device__ __forceinline__ uint32_t codes_to_e2m1(uint32_t x) {
+  const uint32_t nz = ~x & 0x11111111u;                 // code is 0 or 2: weight non-zero
+  const uint32_t neg = ~x & ~(x >> 1) & 0x11111111u;    // code is 0: weight -1
+  return (nz << 1) | (neg << 3);
+}
+
+// 16 weights -> one 16-byte e2m1 group in the padded shared-memory form the
+// f8f6f4 MMA reads: 16 nibbles (even k low) in the first 8 bytes, 8 zero bytes.
+__device__ __forceinline__ uint4 unpack16_e2m1(uint32_t w) {
+  uint4 o;
+  o.x = codes_to_e2m1(codes_lo(w));
+  o.y = codes_to_e2m1(codes_hi(w));
+  o.z = 0u;
+  o.w = 0u;
+  return o;
+}
+
+// --------------------------------------------------------- status words
+__device__ __forceinline__ void report_status(int* status, int code) {
+  if (status) atomicOr(status, code);
+}
+
+}  // namespace blt

@@ -1,0 +1,52 @@
+// Internal launchers behind the C ABI (host side). Arguments are already
+// validated by the entry points in api.cu.
+#pragma once
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+#include "../../include/bitlinear.h"
+
+namespace blt {
+
+cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, int64_t K,
+                             int64_t ldx, int mode, void* q, float* xs, cudaStream_t s);
+cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int64_t k,
+                           int8_t* q, float* xs, uint8_t* mask, cudaStream_t s);
+cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
+                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
+                            float* scale, cudaStream_t s);
+
+// Epilogue of the GEMM kernels.
+enum OutMode : int { kOutBf16 = 0, kOutRaw = 1 };
+
+struct GemmArgs {
+  const void* xq;        // int8 codes [M x K] or packed e2m1 [M x K/2]
+  const float* xs;       // [M] (bf16 output only)
+  const uint8_t* Wp;     // [N x K/4]
+  const float* gamma;    // [G] (bf16 output only)
+  int G;
+  int group_end[8];
+  int64_t M, N, K;
+  void* out;             // bf16 [M x ldo] or raw int32/f32 [M x ldo]
+  int64_t ldo;
+  int out_mode;
+  int* status;
+  uint64_t timeout_ns;
+};
+
+// fp4 selects e2m1 activations (f8f6f4 kind, fp32 accumulate); otherwise int8.
+// Returns a CUDA error, or cudaErrorNotSupported when the tensor-map
+// encoder is unavailable (message in *why).
+cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why);
+cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why);
+cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s);
+
+// Driver entry point for cuTensorMapEncodeTiled, resolved once at run time.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn get_encode_tiled();
+int num_sms();
+
+}  // namespace blt

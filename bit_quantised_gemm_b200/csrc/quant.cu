@@ -1,0 +1,384 @@
+// Per-token activation quantisers, top-k sparsifier and KV-cache quantiser.
+//
+// All three are HBM-bound: one pass reads the bf16 rows once (16-byte
+// vector loads), reductions run in registers / shared memory, codes are
+// written once with vector stores. No fast-math: every scale and rounding is
+// an IEEE fp32 operation (explicit __fdiv_rn / __fmul_rn, rintf = RNE).
+#include "common.cuh"
+#include "launch.h"
+
+namespace blt {
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float block_max_256(float v, float* red /*[8]*/) {
+  v = warp_max(v);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int i = 1; i < kQuantThreads / 32; ++i) r = fmaxf(r, red[i]);
+  __syncthreads();
+  return r;
+}
+
+// Inclusive prefix sum over the 256 threads of the block.
+__device__ __forceinline__ uint32_t block_scan_256(uint32_t v, uint32_t* sums /*[8]*/) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) sums[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t s = lane < 8 ? sums[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < 8; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += n;
+    }
+    if (lane < 8) sums[lane] = s;
+  }
+  __syncthreads();
+  if (wid > 0) v += sums[wid - 1];
+  __syncthreads();
+  return v;
+}
+
+__device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi) {
+  return static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(h, inv)), lo), hi));
+}
+
+__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+// 8 fp32 -> 8 e2m1 nibbles (even index low), round to nearest even, satfinite.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(out)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return out;
+}
+
+// ------------------------------------------------------------ quant_act
+// One block per token row. Pass 1 loads the row (and the up row for the
+// ReLU^2 gate), keeps h in shared memory and reduces the absmax; pass 2
+// writes the codes.
+template <int MODE, bool RELU2>
+__global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int K, int64_t ldx,
+    void* __restrict__ q_out, float* __restrict__ xs_out) {
+  extern __shared__ float4 s_row4[];
+  float* s_row = reinterpret_cast<float*>(s_row4);
+  __shared__ float red[kQuantThreads / 32];
+  const int64_t m = blockIdx.x;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + m * ldx);
+  const uint4* ur = reinterpret_cast<const uint4*>(RELU2 ? up + m * ldx : x);
+  const int nchunk = K >> 3;
+
+  float amax = 0.f;
+  for (int c = threadIdx.x; c < nchunk; c += kQuantThreads) {
+    float h[8];
+    bf16x8_to_f32(__ldg(xr + c), h);
+    if (RELU2) {
+      float u[8];
+      bf16x8_to_f32(__ldg(ur + c), u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float r = h[i] > 0.f ? h[i] : 0.f;
+        h[i] = __fmul_rn(__fmul_rn(r, r), u[i]);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(h[i]));
+    s_row4[2 * c] = make_float4(h[0], h[1], h[2], h[3]);
+    s_row4[2 * c + 1] = make_float4(h[4], h[5], h[6], h[7]);
+  }
+  amax = block_max_256(amax, red);  // also orders the shared-memory row
+
+  constexpr float Q = MODE == BITLINEAR_MODE_INT8 ? 127.f : (MODE == BITLINEAR_MODE_INT4 ? 7.f : 6.f);
+  const float a = fmaxf(amax, kEps);
+  const float inv = __fdiv_rn(Q, a);
+  if (threadIdx.x == 0) xs_out[m] = __fdiv_rn(a, Q);
+
+  for (int c = threadIdx.x; c < nchunk; c += kQuantThreads) {
+    const float4 p0 = s_row4[2 * c], p1 = s_row4[2 * c + 1];
+    const float h[8] = {p0.x, p0.y, p0.z, p0.w, p1.x, p1.y, p1.z, p1.w};
+    if (MODE == BITLINEAR_MODE_FP4) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(h[i], inv);
+      reinterpret_cast<uint32_t*>(q_out)[m * (K >> 3) + c] = cvt_e2m1x8(v);
+    } else {
+      int q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = quant_code(h[i], inv, -Q - 1.f, Q);
+      reinterpret_cast<uint2*>(q_out)[m * (K >> 3) + c] =
+          make_uint2(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]));
+    }
+  }
+  (void)s_row;
+}
+
+template <int MODE, bool RELU2>
+static cudaError_t launch_quant_t(const uint16_t* x, const uint16_t* up, int64_t M, int K,
+                                  int64_t ldx, void* q, float* xs, cudaStream_t s) {
+  const size_t smem = static_cast<size_t>(K) * sizeof(float);
+  auto kern = quant_act_kernel<MODE, RELU2>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+  }
+  kern<<<static_cast<unsigned>(M), kQuantThreads, smem, s>>>(x, up, K, ldx, q, xs);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, int64_t K,
+                             int64_t ldx, int mode, void* q, float* xs, cudaStream_t s) {
+  const int k = static_cast<int>(K);
+  if (up) {
+    if (mode == BITLINEAR_MODE_INT8) return launch_quant_t<BITLINEAR_MODE_INT8, true>(x, up, M, k, ldx, q, xs, s);
+    if (mode == BITLINEAR_MODE_INT4) return launch_quant_t<BITLINEAR_MODE_INT4, true>(x, up, M, k, ldx, q, xs, s);
+    return launch_quant_t<BITLINEAR_MODE_FP4, true>(x, up, M, k, ldx, q, xs, s);
+  }
+  if (mode == BITLINEAR_MODE_INT8) return launch_quant_t<BITLINEAR_MODE_INT8, false>(x, up, M, k, ldx, q, xs, s);
+  if (mode == BITLINEAR_MODE_INT4) return launch_quant_t<BITLINEAR_MODE_INT4, false>(x, up, M, k, ldx, q, xs, s);
+  return launch_quant_t<BITLINEAR_MODE_FP4, false>(x, up, M, k, ldx, q, xs, s);
+}
+
+// ----------------------------------------------------------------- top-k
+// One block per row; thread t owns the contiguous elements [t*E, t*E+E).
+// Radix select on the 15-bit |bf16| key: an 8-bit histogram of key >> 7,
+// then a 7-bit histogram of the low bits inside the selected bin, gives the
+// threshold key T and the count of keys above it. Keys equal to T are kept
+// in column order until k are kept (a block prefix sum gives each thread's
+// starting rank among the equal keys).
+template <int E>
+__global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
+    const uint16_t* __restrict__ x, int K, int64_t ldx, int k, int8_t* __restrict__ q_out,
+    float* __restrict__ xs_out, uint8_t* __restrict__ mask_out) {
+  __shared__ uint32_t hist[256];
+  __shared__ uint32_t sums[8];
+  __shared__ float red[8];
+  __shared__ uint32_t sel[2];  // selected bin, count of keys above the bin
+  const int t = threadIdx.x;
+  const int64_t m = blockIdx.x;
+  const int base = t * E;
+  const int nvalid = max(0, min(E, K - base));  // multiple of 8
+
+  uint16_t v[E];
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) {
+    uint4 w = make_uint4(0, 0, 0, 0);
+    if (c * 8 < nvalid) w = __ldg(reinterpret_cast<const uint4*>(x + m * ldx + base) + c);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[c * 8 + 2 * i] = static_cast<uint16_t>(ws[i] & 0xFFFFu);
+      v[c * 8 + 2 * i + 1] = static_cast<uint16_t>(ws[i] >> 16);
+    }
+  }
+
+  // pass 1: high 8 bits of the key
+  hist[t] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < E; ++i)
+    if (i < nvalid) atomicAdd(&hist[(v[i] & 0x7FFF) >> 7], 1u);
+  __syncthreads();
+  {
+    const uint32_t c = hist[255 - t];
+    const uint32_t s = block_scan_256(c, sums);  // keys in bins >= 255 - t
+    if (s >= static_cast<uint32_t>(k) && s - c < static_cast<uint32_t>(k)) {
+      sel[0] = 255 - t;
+      sel[1] = s - c;
+    }
+  }
+  __syncthreads();
+  const uint32_t b1 = sel[0], above1 = sel[1];
+  __syncthreads();
+
+  // pass 2: low 7 bits inside bin b1
+  hist[t] = 0u;
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const uint32_t key = v[i] & 0x7FFF;
+    if (i < nvalid && (key >> 7) == b1) atomicAdd(&hist[key & 127], 1u);
+  }
+  __syncthreads();
+  {
+    const uint32_t c = t < 128 ? hist[127 - t] : 0u;
+    const uint32_t s = block_scan_256(c, sums);
+    const uint32_t need = static_cast<uint32_t>(k) - above1;
+    if (t < 128 && s >= need && s - c < need) {
+      sel[0] = 127 - t;
+      sel[1] = s - c;
+    }
+  }
+  __syncthreads();
+  const uint32_t T = (b1 << 7) | sel[0];
+  const uint32_t need_eq = static_cast<uint32_t>(k) - above1 - sel[1];  // >= 1
+
+  // pass 3: rank of equal keys in column order
+  uint32_t n_eq = 0;
+#pragma unroll
+  for (int i = 0; i < E; ++i) n_eq += (i < nvalid && (v[i] & 0x7FFF) == T) ? 1u : 0u;
+  uint32_t rank = block_scan_256(n_eq, sums) - n_eq;  // exclusive prefix
+
+  uint32_t keep_bits[(E + 31) / 32];
+#pragma unroll
+  for (int j = 0; j < (E + 31) / 32; ++j) keep_bits[j] = 0u;
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < E; ++i) {
+    const uint32_t key = v[i] & 0x7FFF;
+    bool keep = false;
+    if (i < nvalid) {
+      if (key > T) keep = true;
+      else if (key == T) { keep = rank < need_eq; ++rank; }
+    }
+    if (keep) {
+      keep_bits[i >> 5] |= 1u << (i & 31);
+      amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16)));
+    }
+  }
+  amax = block_max_256(amax, red);
+  const float a = fmaxf(amax, kEps);
+  const float inv = __fdiv_rn(127.f, a);
+  if (t == 0) xs_out[m] = __fdiv_rn(a, 127.f);
+
+#pragma unroll
+  for (int c = 0; c < E / 8; ++c) {
+    if (c * 8 < nvalid) {
+      int q[8];
+      uint32_t mb = 0u;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int idx = c * 8 + i;
+        const bool kp = (keep_bits[idx >> 5] >> (idx & 31)) & 1u;
+        const float xv = __uint_as_float(static_cast<uint32_t>(v[idx]) << 16);
+        q[i] = kp ? quant_code(xv, inv, -128.f, 127.f) : 0;
+        mb |= (kp ? 1u : 0u) << i;
+      }
+      reinterpret_cast<uint2*>(q_out + m * K + base)[c] =
+          make_uint2(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]));
+      if (mask_out) mask_out[m * (K >> 3) + (base >> 3) + c] = static_cast<uint8_t>(mb);
+    }
+  }
+}
+
+cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int64_t k,
+                           int8_t* q, float* xs, uint8_t* mask, cudaStream_t s) {
+  const int kk = static_cast<int>(k), KK = static_cast<int>(K);
+  const unsigned grid = static_cast<unsigned>(M);
+  if (K <= 8 * kQuantThreads)
+    topk_i8_kernel<8><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
+  else if (K <= 16 * kQuantThreads)
+    topk_i8_kernel<16><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
+  else if (K <= 32 * kQuantThreads)
+    topk_i8_kernel<32><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
+  else
+    topk_i8_kernel<64><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ KV 3-bit
+// Each thread quantises 8 consecutive head dims (one 16-byte load); the
+// G = D/8 threads of one (token, head) row reduce their absmax with a
+// segmented warp shuffle. A warp covers 32/G whole rows whose 3-bit
+// streams (3 bytes per thread) form 96 contiguous bytes, staged in shared
+// memory and written as 24 aligned words.
+template <int G>
+__global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
+    const uint16_t* __restrict__ kv, int64_t rows, int64_t H, const int32_t* __restrict__ keep4,
+    int n4, uint8_t* __restrict__ codes3, uint8_t* __restrict__ codes4, float* __restrict__ scale) {
+  constexpr int D = 8 * G;
+  __shared__ __align__(16) uint8_t stage[kQuantThreads / 32][96];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
+  const int64_t row = gtid / G;
+  const int g = static_cast<int>(gtid % G);
+  const bool valid = row < rows;
+
+  float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (valid) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kv + row * D) + g), f);
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+  for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+
+  const int64_t t = row / H, h = row % H;
+  int j = -1;  // index of t among the 4-bit tokens
+  if (valid) {
+    int lo = 0, hi = n4 - 1;
+    while (lo <= hi) {
+      const int mid = (lo + hi) >> 1;
+      const int p = __ldg(keep4 + mid);
+      if (p == t) { j = mid; break; }
+      if (p < t) lo = mid + 1; else hi = mid - 1;
+    }
+  }
+  const bool four = j >= 0;
+  const float Q = four ? 7.f : 3.f;
+  const float a = fmaxf(amax, kEps);
+  const float inv = __fdiv_rn(Q, a);
+  const float lo_c = four ? -8.f : -4.f, hi_c = four ? 7.f : 3.f;
+  uint32_t packed3 = 0u, packed4 = 0u;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int c = quant_code(f[i], inv, lo_c, hi_c);
+    packed3 |= static_cast<uint32_t>(c + 4) << (3 * i);
+    packed4 |= static_cast<uint32_t>(c + 8) << (4 * i);
+  }
+  if (four) packed3 = 0u;
+  if (valid && four)
+    reinterpret_cast<uint32_t*>(codes4 + (static_cast<int64_t>(j) * H + h) * (D / 2))[g] = packed4;
+  if (valid && g == 0) scale[row] = __fdiv_rn(a, Q);
+
+  stage[wid][3 * lane + 0] = static_cast<uint8_t>(packed3);
+  stage[wid][3 * lane + 1] = static_cast<uint8_t>(packed3 >> 8);
+  stage[wid][3 * lane + 2] = static_cast<uint8_t>(packed3 >> 16);
+  __syncwarp();
+  const int64_t warp_row0 = (gtid - lane) / G;
+  const int64_t rows_here = rows - warp_row0;
+  const int nbytes = rows_here >= 32 / G ? 96 : static_cast<int>(rows_here > 0 ? rows_here : 0) * 3 * G;
+  if (lane * 4 < nbytes)
+    reinterpret_cast<uint32_t*>(codes3 + warp_row0 * (3 * G))[lane] =
+        reinterpret_cast<const uint32_t*>(stage[wid])[lane];
+}
+
+cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
+                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
+                            float* scale, cudaStream_t s) {
+  const int64_t rows = T * H;
+  const int G = static_cast<int>(D / 8);
+  const int64_t threads = rows * G;
+  const unsigned grid = static_cast<unsigned>((threads + kQuantThreads - 1) / kQuantThreads);
+  const int n = static_cast<int>(n4);
+  if (G == 8) kv_quant_kernel<8><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
+  else if (G == 16) kv_quant_kernel<16><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
+  else kv_quant_kernel<32><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
+  return cudaGetLastError();
+}
+
+}  // namespace blt

@@ -1,0 +1,112 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+the header declares, the host weight-prep call matches the oracle bit for
+bit, and bad arguments are rejected on the host before any launch."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import bit_quantised_gemm_b200 as B
+from bit_quantised_gemm_b200 import _lib
+from conftest import golden
+from oracle import bitlinear_oracle as O
+import workloads as W
+
+
+def test_library_exports_every_declared_function():
+    L = B.lib()
+    declared = B.header_functions()
+    assert len(declared) >= 14
+    for name in declared:
+        assert hasattr(L, name), name
+    assert set(declared) == set(_lib._SIGS)
+    assert B.version() == 100
+
+
+@pytest.mark.parametrize("K,N,groups,seed", [
+    (256, 256, (256,), 0), (64, 96, (32, 96), 1), (2048, 384, (128, 256, 384), 2),
+    (16, 16, (16,), 3)])
+def test_ternarize_pack_matches_oracle(K, N, groups, seed):
+    Wm = W.weights(np.random.default_rng(seed), K, N)
+    Wp, gamma = B.ternarize_pack(Wm, groups)
+    Wt_o, gamma_o = O.ternarize(Wm, groups)
+    assert np.array_equal(gamma, gamma_o)
+    assert np.array_equal(Wp, O.pack_ternary(Wt_o))
+
+
+def test_ternarize_pack_golden_ties():
+    g = golden("ternarize_ties.txt")
+    for case in "ABC":
+        Wm = np.array([float(v) for v in g[f"W_{case}"]], np.float32).reshape(2, 2)
+        # K must be a multiple of 16: repeat the 2 x 2 block 8 times down K
+        # (the mean |W| and so every code are unchanged)
+        Wp, gamma = B.ternarize_pack(np.tile(Wm, (8, 1)), (2,))
+        Wt = O.unpack_ternary(Wp, 16)
+        want = np.array([int(v) for v in g[f"Wt_{case}"]]).reshape(2, 2)
+        assert np.array_equal(Wt, np.tile(want, (8, 1)))
+
+
+def test_ternarize_pack_golden_layout():
+    g = golden("pack_layout.txt")
+    col = np.array([int(v) for v in g["Wt_col"]], np.float32).reshape(16, 1)
+    # values +-1 with mean |W| = 3/16: +-1/gamma rounds to +-5 -> clamps to +-1
+    Wp, gamma = B.ternarize_pack(col, (1,))
+    assert Wp[0].tolist() == [int(b, 16) for b in g["bytes"]]
+
+
+FAKE = 1 << 20  # a 16-byte aligned non-null address; never dereferenced on a host-side error
+ge1 = np.array([256], np.int64)
+
+
+def _gemm(fn, **kw):
+    a = dict(xq=FAKE, xs=FAKE, Wp=FAKE, gamma=FAKE, ge=ge1.ctypes.data, G=1, M=16, N=256, K=256,
+             y=FAKE, ldy=256)
+    a.update(kw)
+    return getattr(B.lib(), fn)(a["xq"], a["xs"], a["Wp"], a["gamma"], a["ge"], a["G"], a["M"],
+                                a["N"], a["K"], a["y"], a["ldy"], None, None)
+
+
+@pytest.mark.parametrize("fn", ["bitlinear_gemm_w2a8", "bitlinear_gemm_w2a4",
+                                "bitlinear_gemm_w2fp4", "bitlinear_gemv_w2"])
+def test_gemm_argument_errors(fn):
+    assert _gemm(fn, K=200) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, N=250) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, M=-1) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, xq=None) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, xq=FAKE + 4) == _lib.ERR_ALIGNMENT
+    assert _gemm(fn, ldy=100) == _lib.ERR_INVALID_ARG
+    bad = np.array([100, 200], np.int64)
+    assert _gemm(fn, ge=bad.ctypes.data, G=2) == _lib.ERR_INVALID_ARG  # last end != N
+    dec = np.array([200, 100, 256], np.int64)
+    assert _gemm(fn, ge=dec.ctypes.data, G=3) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, G=9) == _lib.ERR_INVALID_ARG
+    assert _gemm(fn, M=0) == _lib.OK  # empty: nothing launched
+
+
+def test_gemv_and_fp4_specific_limits():
+    assert _gemm("bitlinear_gemv_w2", M=65) == _lib.ERR_INVALID_ARG
+    assert _gemm("bitlinear_gemm_w2fp4", K=192) == _lib.ERR_INVALID_ARG  # K % 128
+
+
+def test_quantiser_argument_errors():
+    L = B.lib()
+    assert L.bitlinear_quant_act(FAKE, None, 4, 250, 256, 0, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(FAKE, None, 4, 256, 256, 7, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(FAKE, None, 4, 256, 100, 0, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.bitlinear_quant_act(FAKE + 2, None, 4, 256, 256, 0, FAKE, FAKE, None) == _lib.ERR_ALIGNMENT
+    assert L.bitlinear_quant_act(FAKE, None, 0, 256, 256, 0, FAKE, FAKE, None) == _lib.OK
+    assert L.bitlinear_topk_sparsify_i8(FAKE, 4, 32768, 32768, 0, FAKE, FAKE, None, None) == _lib.ERR_UNSUPPORTED
+    assert L.bitlinear_topk_sparsify_i8(FAKE, 4, 256, 256, -1, FAKE, FAKE, None, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_quant_3bit(FAKE, 4, 2, 96, None, 0, FAKE, None, FAKE, None) == _lib.ERR_UNSUPPORTED
+    assert L.kv_quant_3bit(FAKE, 4, 2, 128, None, 1, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_quant_3bit(FAKE, 0, 2, 128, None, 0, FAKE, None, FAKE, None) == _lib.OK
+    assert L.bitlinear_set_wait_timeout_ns(0) == _lib.ERR_INVALID_ARG
+    msg = L.bitlinear_last_error().decode()
+    assert "timeout" in msg
+
+
+def test_error_raises_python_exception():
+    with pytest.raises(B.BitlinearError) as ei:
+        B.set_wait_timeout_ns(-5)
+    assert ei.value.code == _lib.ERR_INVALID_ARG
+    B.set_wait_timeout_ns(2_000_000_000)

@@ -1,0 +1,246 @@
+"""GPU parity: every C-ABI entry point against the CPU oracle on the same
+seeded inputs. Integer work (codes, masks, int32 accumulators, packed bytes)
+must match bit for bit; bf16 outputs within 2 bf16 ulp; FP4 fp32
+accumulators within 1e-5 relative (they are exact in practice)."""
+import numpy as np
+import pytest
+import torch
+
+import bit_quantised_gemm_b200 as B
+from oracle import bitlinear_oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+BF16_ULP_TOL = 2
+FP4_REL_TOL = 1e-5
+DEV = "cuda:0"
+
+
+def dev_bf16(bits: np.ndarray) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def host(t: torch.Tensor) -> np.ndarray:
+    return t.cpu().numpy()
+
+
+def bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def assert_bf16_close(got_bits, want_bits, tol=BF16_ULP_TOL):
+    d = O.bf16_ulp_diff(got_bits, want_bits)
+    assert d.max() <= tol, f"max ulp diff {d.max()} at {np.unravel_index(d.argmax(), d.shape)}"
+
+
+@pytest.fixture(autouse=True)
+def _clean_status():
+    B.status_buffer().zero_()
+    yield
+    B.check_status()
+
+
+# ----------------------------------------------------------- quantisers
+@pytest.mark.parametrize("mode", [O.MODE_INT8, O.MODE_INT4, O.MODE_FP4])
+@pytest.mark.parametrize("M,K", [(1, 256), (17, 2048), (130, 4096 + 128), (3, 11008)])
+@pytest.mark.parametrize("relu2", [False, True])
+def test_quant_act_parity(mode, M, K, relu2):
+    rng = np.random.default_rng(M * K + mode)
+    x = W.student_t_bf16(rng, M, K)
+    up = W.normal_bf16(rng, (M, K)) if relu2 else None
+    q, xs = B.quant_act(dev_bf16(x), mode, up=dev_bf16(up) if relu2 else None)
+    q_o, xs_o = O.quant_act(x, mode, up)
+    assert np.array_equal(host(xs), xs_o)
+    assert np.array_equal(host(q).view(np.uint8), q_o.view(np.uint8))
+
+
+def test_quant_act_strided_rows_and_zero_row():
+    rng = np.random.default_rng(5)
+    x = W.normal_bf16(rng, (9, 512))
+    x[4] = 0
+    xt = dev_bf16(x)[:, :384]  # row stride 512, K = 384
+    for mode in (O.MODE_INT8, O.MODE_INT4, O.MODE_FP4):
+        q, xs = B.quant_act(xt, mode)
+        q_o, xs_o = O.quant_act(np.ascontiguousarray(x[:, :384]), mode)
+        assert np.array_equal(host(xs), xs_o)
+        assert np.array_equal(host(q).view(np.uint8), q_o.view(np.uint8))
+
+
+def test_fp4_rounding_midpoints():
+    """Rows whose absmax is 6 (scale 1): every e2m1 midpoint and its bf16
+    neighbours, both signs, and signed zeros."""
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    vals = []
+    for m in mids:
+        b = O.f32_to_bf16(np.float32(m))
+        vals += [m, float(O.bf16_to_f32(b + 1)), float(O.bf16_to_f32(b - 1))]
+    vals += [0.0, -0.0, 0.1, -0.1, 6.0, 4.0, 3.0]
+    vals += [-v for v in vals]
+    row = np.array(vals + [0.0] * (-len(vals) % 16), np.float32)
+    row[0] = 6.0
+    x = O.f32_to_bf16(np.stack([row, row * np.float32(0.5)]))
+    q, xs = B.quant_act(dev_bf16(x), O.MODE_FP4)
+    q_o, xs_o = O.quant_act(x, O.MODE_FP4)
+    assert np.array_equal(host(q), q_o)
+    assert np.array_equal(host(xs), xs_o)
+
+
+@pytest.mark.parametrize("K", [64, 256, 4096, 11008, 16384])
+@pytest.mark.parametrize("k", [0, 1, 7, None])
+def test_topk_parity(K, k):
+    rng = np.random.default_rng(K + (k or 0))
+    M = 19
+    xf = rng.standard_t(3, size=(M, K)).astype(np.float32)
+    xf[1] = np.round(xf[1] * 2) / 2        # heavy ties
+    xf[2] = 1.0                            # all equal
+    xf[3] = 0.0                            # all zero
+    x = O.f32_to_bf16(xf)
+    kk = K if k is None else k
+    q, xs, mask = B.topk_sparsify_i8(dev_bf16(x), k=kk, mask=True)
+    q_o, xs_o, m_o = O.topk_sparsify_i8(x, kk if kk else 0)
+    assert np.array_equal(host(mask), O.pack_mask_bits(m_o))
+    assert np.array_equal(host(q), q_o)
+    assert np.array_equal(host(xs), xs_o)
+
+
+def test_topk_full_size_o_proj():
+    d = W.o_proj_sparse(make_weights=False, M=1024)  # the o_proj input recipe, 1024 rows
+    q, xs, mask = B.topk_sparsify_i8(dev_bf16(d["x"]), mask=True)
+    q_o, xs_o, m_o = O.topk_sparsify_i8(d["x"])
+    assert np.array_equal(host(q), q_o) and np.array_equal(host(xs), xs_o)
+    assert np.array_equal(host(mask), O.pack_mask_bits(m_o))
+
+
+@pytest.mark.parametrize("D", [64, 128, 256])
+@pytest.mark.parametrize("keep", [(0,), (0, 5, 6, 37), ()])
+def test_kv_quant_parity(D, keep):
+    rng = np.random.default_rng(D + len(keep))
+    T, H = 41, 3
+    kv = W.normal_bf16(rng, (T, H, D))
+    kv[7, 1] = 0  # an all-zero head row
+    kp = torch.tensor(keep, dtype=torch.int32, device=DEV) if keep else None
+    c3, c4, s = B.kv_quant_3bit(dev_bf16(kv), kp)
+    c3_o, c4_o, s_o = O.kv_quant_3bit(kv, keep)
+    assert np.array_equal(host(s), s_o)
+    assert np.array_equal(host(c3), c3_o)
+    if keep:
+        assert np.array_equal(host(c4), c4_o)
+
+
+# ------------------------------------------------------------------ GEMMs
+def prep_weights(K, N, groups, seed):
+    Wm = W.weights(np.random.default_rng(seed), K, N)
+    Wt, gamma = O.ternarize(Wm, groups)
+    Wp = O.pack_ternary(Wt)
+    return Wt, gamma, torch.from_numpy(Wp).to(DEV), torch.from_numpy(gamma).to(DEV)
+
+
+GEMM_SHAPES = [  # (M, N, K): single tile, ragged M/N, half k-block, many tiles
+    (16, 256, 256), (1, 16, 64), (130, 272, 320), (257, 512, 1024), (2048, 4096, 256),
+    (300, 768, 2048 + 64)]
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_gemm_int8_accumulators_bit_exact(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    Wt, _, Wp, _ = prep_weights(K, N, (N,), K)
+    acc = B.gemm_w2a8_acc(torch.from_numpy(xq).to(DEV), Wp)
+    B.check_status()
+    assert np.array_equal(host(acc).astype(np.int64), O.gemm_acc_int(xq, Wt))
+
+
+@pytest.mark.parametrize("M,N,K", [s for s in GEMM_SHAPES if s[2] % 128 == 0])
+def test_gemm_fp4_accumulators(M, N, K):
+    rng = np.random.default_rng(M * 3 + N + K)
+    codes = rng.integers(0, 16, size=(M, K)).astype(np.uint8)
+    xf4 = O.pack_nibbles(codes)
+    Wt, _, Wp, _ = prep_weights(K, N, (N,), K + 1)
+    acc = B.gemm_w2fp4_acc(torch.from_numpy(xf4).to(DEV), Wp)
+    B.check_status()
+    want = O.gemm_acc_fp4(codes, Wt)
+    got = host(acc).astype(np.float64)
+    assert np.all(np.abs(got - want) <= FP4_REL_TOL * np.maximum(np.abs(want), 1.0))
+    assert np.array_equal(got, want)  # exact in practice (multiples of 0.5 < 2^24)
+
+
+@pytest.mark.parametrize("mode", [O.MODE_INT8, O.MODE_INT4, O.MODE_FP4])
+@pytest.mark.parametrize("M,N,K,groups", [(16, 256, 256, (256,)), (200, 768, 2048, (256, 512, 768)),
+                                          (129, 1056, 512, (528, 1056))])
+def test_bitlinear_layer_end_to_end(mode, M, N, K, groups):
+    """bf16 X -> quantiser -> GEMM -> bf16 Y, both sides from the same X and W."""
+    rng = np.random.default_rng(M + mode)
+    x = W.outlier_bf16(rng, M, K)[0]
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, groups, 7)
+    xq_o, xs_o = O.quant_act(x, mode)
+    q, xs = B.quant_act(dev_bf16(x), mode)
+    if mode == O.MODE_FP4:
+        y = B.gemm_w2fp4(q, xs, Wp, gamma_d, groups)
+        _, y_o = O.bitlinear_fp4(xq_o, xs_o, Wt, gamma, groups)
+    else:
+        fn = B.gemm_w2a8 if mode == O.MODE_INT8 else B.gemm_w2a4
+        y = fn(q, xs, Wp, gamma_d, groups)
+        _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, groups)
+    B.check_status()
+    assert_bf16_close(bits(y), y_o)
+
+
+@pytest.mark.parametrize("M", [1, 8, 17, 64])
+@pytest.mark.parametrize("N,K", [(128, 128), (4096, 4096), (4096, 11008), (1024, 512)])
+def test_gemv_parity(M, N, K):
+    rng = np.random.default_rng(M + N + K)
+    xq = rng.integers(-128, 128, size=(M, K)).astype(np.int8)
+    xs = rng.uniform(0.01, 1, M).astype(np.float32)
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, (N,), 11)
+    y = B.gemv_w2(torch.from_numpy(xq).to(DEV), torch.from_numpy(xs).to(DEV), Wp, gamma_d, (N,))
+    B.check_status()
+    _, y_o = O.bitlinear_int(xq, xs, Wt, gamma, (N,))
+    assert_bf16_close(bits(y), y_o)
+
+
+def test_gemv_matches_gemm():
+    rng = np.random.default_rng(3)
+    M, N, K = 33, 2048, 2048
+    xq = torch.from_numpy(rng.integers(-8, 8, size=(M, K)).astype(np.int8)).to(DEV)
+    xs = torch.from_numpy(rng.uniform(0.01, 1, M).astype(np.float32)).to(DEV)
+    _, _, Wp, gamma_d = prep_weights(K, N, (1024, 2048), 12)
+    y1 = B.gemv_w2(xq, xs, Wp, gamma_d, (1024, 2048))
+    y2 = B.gemm_w2a4(xq, xs, Wp, gamma_d, (1024, 2048))
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_empty_inputs_are_noops():
+    e = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
+    q, xs = B.quant_act(e, O.MODE_INT8)
+    assert q.shape == (0, 256)
+    _, _, Wp, g = prep_weights(256, 256, (256,), 1)
+    y = B.gemm_w2a8(torch.empty((0, 256), dtype=torch.int8, device=DEV), xs, Wp, g, (256,))
+    assert y.shape == (0, 256)
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    st = torch.zeros(1, dtype=torch.int32, device=DEV)
+    B.debug_wait_timeout(st, 2_000_000)  # 2 ms on a barrier nothing arrives on
+    with pytest.raises(B.BitlinearError) as ei:
+        B.check_status(st)
+    assert ei.value.code == -5
+    assert int(st.item()) == 1
+    # the context is still usable
+    rng = np.random.default_rng(0)
+    xq = rng.integers(-128, 128, size=(32, 256)).astype(np.int8)
+    Wt, _, Wp, _ = prep_weights(256, 256, (256,), 0)
+    acc = B.gemm_w2a8_acc(torch.from_numpy(xq).to(DEV), Wp)
+    assert np.array_equal(host(acc).astype(np.int64), O.gemm_acc_int(xq, Wt))
+
+
+def test_library_prep_feeds_gpu_gemm():
+    """Weights prepared by the library's host call (not the oracle) give the
+    same GEMM result as the oracle's own ternarisation."""
+    d = W.single_w2a4()
+    Wp_l, gamma_l = B.ternarize_pack(d["proj"].W, (256,))
+    Wt, gamma = O.ternarize(d["proj"].W, (256,))
+    q, xs = B.quant_act(dev_bf16(d["x"]), O.MODE_INT4)
+    y = B.gemm_w2a4(q, xs, torch.from_numpy(Wp_l).to(DEV), torch.from_numpy(gamma_l).to(DEV), (256,))
+    xq_o, xs_o = O.quant_act(d["x"], O.MODE_INT4)
+    _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, (256,))
+    assert_bf16_close(bits(y), y_o)
