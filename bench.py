@@ -1,0 +1,651 @@
+#!/usr/bin/env python
+"""Benchmark of the BitLinear hot path on B200.
+
+One step = the input-projection prefill workload, both activation variants:
+  X [2048 tokens x 2048] bf16, N(0,1) with 1% outlier channels x20;
+  fused q|k|v W [2048 x 6144] (3 scale groups) and gate|up W [2048 x 11264]
+  (2 groups), ternary, 2-bit packed.
+  INT4: quant_act(X, INT4) -> gemm_w2a4(qkv) -> gemm_w2a4(gate_up)
+  FP4 : quant_act(X, FP4)  -> gemm_w2fp4(qkv) -> gemm_w2fp4(gate_up)
+value = 2*M*K*N summed over the four GEMMs / step time, in TOPS.
+
+Inputs are already resident in HBM; R replicas of all buffers rotate so the
+working set (>= 270 MB) exceeds the 126 MB L2 between consecutive steps.
+Each replica's step is one CUDA graph. Per-kernel durations come from CUDA
+events captured inside the graphs (last 24 steps of the timed region).
+
+Also reported (same run, rank 0, unless --no-breakdown): the o_proj top-k
+INT8 GEMM, the down_proj ReLU^2 INT8 GEMM, the decode layer at batch 1/8/64
+(weight GB/s) and the 3-bit KV quantiser (GB/s).
+
+--impl reference times the CPU oracle on host cores on a bounded sample of
+the same workload (rows of X), in the same metric.
+
+Multi-GPU (torchrun): each rank runs the same per-GPU workload (replicas,
+weak scaling, no collective on the data path); value = all ranks' ops /
+max-over-ranks time.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "BitLinear prefill TOPS vs int8/fp4 peak; decode weight GB/s vs HBM (1×B200)"
+WORKLOAD = ("Input-projection prefill W1.58A4: X [2048 tokens×2048] bf16 ~N(0,1) with 1% "
+            "channels ×20 outliers; fused q/k/v W [2048×6144] and gate/up W "
+            "[2048×2×5632] ternary; INT4 and FP4(e2m1) activation variants")
+M_TOK, D, FFN = 2048, 2048, 5632
+QKV = (D, (D, 2 * D, 3 * D))
+GU = (D, (FFN, 2 * FFN))
+OPS_PER_STEP = 2 * (2 * M_TOK * D * 3 * D + 2 * M_TOK * D * 2 * FFN)
+# nominal dense ratios to bf16 (2.25 PF): int8 4.5 P, fp8 4.5 P, fp4 9 P
+RATIO_INT8, RATIO_FP4 = 2.0, 4.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+GEMM_SRC = os.path.join(ROOT, "bit_quantised_gemm_b200", "csrc", "gemm.cu")
+# DRAM bytes per launch of the INT4-path qkv GEMM from one ncu capture, with
+# the sha256 of the kernel source it was taken on (null once it changes).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_w2a4_qkv_prefill_2048x2048x6144.md")
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=1000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-breakdown", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--seed", type=int, default=1)
+    return ap.parse_args()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def read_traffic():
+    """(bytes per launch, source) from the committed ncu summary, or (None, why)."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None, "no ncu capture committed"
+    text = open(TRAFFIC_FILE).read()
+    src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
+    vals = {}
+    for line in text.splitlines():
+        if line.startswith("traffic_bytes_per_launch:"):
+            vals["t"] = float(line.split(":", 1)[1])
+        if line.startswith("kernel_source_sha256:"):
+            vals["h"] = line.split(":", 1)[1].strip()
+    if "t" not in vals or vals.get("h") != src_hash:
+        return None, "kernel changed since the ncu capture"
+    return vals["t"], "ncu"
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples during the timed region (SM clock, throttle reasons)."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.th = threading.Thread(target=self._read, daemon=True)
+            self.th.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.th.join(timeout=2)
+        sm, smax, reasons, util = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                util.append(float(parts[4]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [s for s, u in zip(sm, util) if u > 0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------ distributed
+def dist_init():
+    import torch
+    import torch.distributed as dist
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1 and not dist.is_initialized():
+        import datetime
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def max_over_ranks(v: float, ws: int) -> float:
+    if ws == 1:
+        return v
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(ws: int):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ our arm
+class PrefillReplica:
+    """Device buffers of one replica of the prefill workload."""
+
+    def __init__(self, B, torch, x_bits, qkv, gu, dev):
+        self.x = torch.from_numpy(x_bits.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.qkv = [torch.from_numpy(a).to(dev) for a in qkv]  # Wp, gamma
+        self.gu = [torch.from_numpy(a).to(dev) for a in gu]
+        M, K = self.x.shape
+        self.q4 = torch.empty((M, K), dtype=torch.int8, device=dev)
+        self.xs4 = torch.empty(M, dtype=torch.float32, device=dev)
+        self.f4 = torch.empty((M, K // 2), dtype=torch.uint8, device=dev)
+        self.xsf = torch.empty(M, dtype=torch.float32, device=dev)
+        self.y = {k: torch.empty((M, n), dtype=torch.bfloat16, device=dev)
+                  for k, n in (("qkv4", 3 * D), ("gu4", 2 * FFN), ("qkvf", 3 * D), ("guf", 2 * FFN))}
+
+
+def run_step(B, r: PrefillReplica, ev=None):
+    """One step; ev (optional) = dict of (start, end) event pairs per GEMM."""
+    def rec(name, i):
+        if ev is not None:
+            ev[name][i].record()
+    B.quant_act(r.x, B.MODE_INT4, out=r.q4, xs=r.xs4)
+    rec("w2a4_qkv", 0); B.gemm_w2a4(r.q4, r.xs4, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkv4"]); rec("w2a4_qkv", 1)
+    rec("w2a4_gu", 0); B.gemm_w2a4(r.q4, r.xs4, r.gu[0], r.gu[1], GU[1], y=r.y["gu4"]); rec("w2a4_gu", 1)
+    B.quant_act(r.x, B.MODE_FP4, out=r.f4, xs=r.xsf)
+    rec("w2fp4_qkv", 0); B.gemm_w2fp4(r.f4, r.xsf, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkvf"]); rec("w2fp4_qkv", 1)
+    rec("w2fp4_gu", 0); B.gemm_w2fp4(r.f4, r.xsf, r.gu[0], r.gu[1], GU[1], y=r.y["guf"]); rec("w2fp4_gu", 1)
+
+
+LAUNCHES_PER_STEP = 6
+GEMM_NAMES = ("w2a4_qkv", "w2a4_gu", "w2fp4_qkv", "w2fp4_gu")
+GEMM_OPS = {"w2a4_qkv": 2 * M_TOK * D * 3 * D, "w2a4_gu": 2 * M_TOK * D * 2 * FFN,
+            "w2fp4_qkv": 2 * M_TOK * D * 3 * D, "w2fp4_gu": 2 * M_TOK * D * 2 * FFN}
+
+
+def make_prefill(B, torch, dev, seed, with_oracle_inputs=False):
+    import workloads as W
+    d = W.input_projection_prefill(seed=seed)
+    qkv_p, gu_p = d["projs"]
+    qkv = B.ternarize_pack(qkv_p.W, qkv_p.group_ends)
+    gu = B.ternarize_pack(gu_p.W, gu_p.group_ends)
+    return d, qkv, gu
+
+
+def graph_set(torch, stream, steps_fns, names, E):
+    """Capture E copies of each replica's step as CUDA graphs, each copy with
+    its own external timing events around the named launches."""
+    graphs, events = [], []
+    with torch.cuda.stream(stream):
+        for fn in steps_fns:  # run once eagerly (first-call set-up outside capture)
+            fn(None)
+    torch.cuda.synchronize()
+    for _ in range(E):
+        for fn in steps_fns:
+            ev = {n: (torch.cuda.Event(enable_timing=True, external=True),
+                      torch.cuda.Event(enable_timing=True, external=True)) for n in names}
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn(ev)
+            graphs.append(g)
+            events.append(ev)
+    torch.cuda.synchronize()
+    return graphs, events
+
+
+def run_graphs(torch, stream, graphs, events, names, steps, warmup, ws=1, clocks=None):
+    """Replay `steps` graphs (rotating) in one timed region; returns (max-over-
+    ranks ms for all steps, {name: mean ms per launch over the last steps})."""
+    NG = len(graphs)
+    for i in range(warmup):
+        graphs[i % NG].replay()
+    torch.cuda.synchronize()
+    if clocks is not None:
+        clocks.start()
+        time.sleep(0.3)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    off = (NG - steps % NG) % NG  # the last NG steps replay every graph once
+    with torch.cuda.stream(stream):
+        t0.record()
+        for i in range(steps):
+            graphs[(i + off) % NG].replay()
+        t1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    clk = clocks.stop() if clocks is not None else None
+    ms = max_over_ranks(t0.elapsed_time(t1), ws)
+    last = min(steps, NG)
+    kms = {}
+    for n in names:
+        v = [events[j][n][0].elapsed_time(events[j][n][1]) for j in range(NG - last, NG)]
+        kms[n] = statistics.mean(v)
+    return ms, kms, clk
+
+
+def bench_ours(args, ws, rank, local):
+    import torch
+    import bit_quantised_gemm_b200 as B
+    dev = f"cuda:{local}"
+    torch.cuda.set_device(local)
+    B.lib()
+    d, qkv, gu = make_prefill(B, torch, dev, args.seed)
+    R = 3
+    reps = [PrefillReplica(B, torch, d["x"], qkv, gu, dev) for _ in range(R)]
+    stream = torch.cuda.Stream(device=dev)
+    fns = [(lambda ev, r=r: run_step(B, r, ev)) for r in reps]
+    graphs, events = graph_set(torch, stream, fns, GEMM_NAMES, E=8)
+    B.check_status(stream=stream)
+    ms, kms, clk = run_graphs(torch, stream, graphs, events, GEMM_NAMES, args.steps, args.warmup,
+                              ws, ClockSampler(local))
+    B.check_status(stream=stream)
+    del graphs
+
+    peaks, peak_src = load_peaks()
+    int8_peak = RATIO_INT8 * peaks["bf16_tflops"]
+    fp4_peak = RATIO_FP4 * peaks["bf16_tflops"]
+    ach = GEMM_OPS["w2a4_qkv"] / (kms["w2a4_qkv"] * 1e-3) / 1e12
+    traffic, tsrc = read_traffic()
+    roofline = {"bound": "tensor", "kernel": "gemm_w2a4 qkv (tcgen05 kind::i8)",
+                "achieved": round(ach, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
+                "frac": round(ach / int8_peak, 4), "traffic": traffic, "traffic_source": tsrc,
+                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TF/s x {RATIO_INT8} "
+                               "(nominal int8/bf16 dense ratio)"}
+    kernels = {}
+    for n in GEMM_NAMES:
+        tops = GEMM_OPS[n] / (kms[n] * 1e-3) / 1e12
+        pk = int8_peak if "w2a4" in n else fp4_peak
+        kernels[n] = {"us": round(kms[n] * 1e3, 2), "TOPS": round(tops, 1),
+                      "frac_of_peak": round(tops / pk, 4),
+                      "peak": "int8" if "w2a4" in n else "fp4 (the f8f6f4 kind runs at the fp8 rate: 0.5 at most)"}
+
+    value = OPS_PER_STEP * args.steps * ws / (ms * 1e-3) / 1e12
+    out = {"metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": ws,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "s8,e2m1 (x ternary)", "data": "synthetic",
+           "config": {"workload": WORKLOAD, "tokens": M_TOK, "d_model": D, "qkv_out": 3 * D,
+                      "gate_up_out": 2 * FFN, "variants": ["INT4 (s8 MMA)", "FP4 e2m1 (f8f6f4 MMA)"],
+                      "parallelism": f"replicas x{ws}",
+                      "l2": f"{R} rotating replicas of all inputs/weights/outputs (>270 MB > 126 MB L2)",
+                      "graphs": "one CUDA graph per step"},
+           "roofline": roofline, "kernels": kernels, "clocks": clk,
+           "gpu_launches": LAUNCHES_PER_STEP * args.steps}
+    return out, (d, qkv, gu, reps, B, torch, dev, stream)
+
+
+def bench_e2e(args, ctx, ws):
+    """Same metric through the Python API with host buffers: per step the
+    H2D copy of X from pinned memory, the six calls, and the D2H copies of
+    the four outputs are inside the timed region."""
+    d, qkv, gu, reps, B, torch, dev, stream = ctx
+    r = reps[0]
+    x_host = torch.from_numpy(d["x"].view(np.int16)).view(torch.bfloat16).pin_memory()
+    outs = {k: torch.empty(v.shape, dtype=v.dtype, pin_memory=True) for k, v in r.y.items()}
+    steps = args.steps
+    h2d = x_host.numel() * 2
+    d2h = sum(v.numel() * 2 for v in outs.values())
+    with torch.cuda.stream(stream):
+        for _ in range(max(1, args.warmup // 4)):
+            r.x.copy_(x_host, non_blocking=True)
+            run_step(B, r)
+            for k, v in outs.items():
+                v.copy_(r.y[k], non_blocking=True)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        t0.record()
+        for _ in range(steps):
+            r.x.copy_(x_host, non_blocking=True)
+            run_step(B, r)
+            for k, v in outs.items():
+                v.copy_(r.y[k], non_blocking=True)
+        t1.record()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = max_over_ranks(t0.elapsed_time(t1), ws)
+    B.check_status(stream=stream)
+    return {"value": round(OPS_PER_STEP * steps * ws / (ms * 1e-3) / 1e12, 3), "unit": "TOPS",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": round(ms / steps, 4), "path": "python API (ctypes -> C ABI), pinned host buffers"}
+
+
+# ------------------------------------------------------- CPU oracle timing
+def _window(wt, c0, width):
+    """Columns [c0, c0+width) of a ternarised projection: (W_t slice, gamma, group ends)."""
+    Wt, gamma, ends = wt
+    c1 = min(c0 + width, Wt.shape[1])
+    g_sub, e_sub, start = [], [], 0
+    for gm, end in zip(gamma, ends):
+        lo, hi = max(start, c0), min(end, c1)
+        if lo < hi:
+            g_sub.append(gm)
+            e_sub.append(hi - c0)
+        start = end
+    return Wt[:, c0:c1], np.array(g_sub, np.float32), tuple(e_sub)
+
+
+def oracle_sample(d, qkv_wt, gu_wt, rows, col0=0, width=None):
+    """Oracle on a sample of the workload: the given token rows through both
+    variants, against a window of `width` output columns of each projection
+    (all of them when width is None). Returns the sample's ops."""
+    from oracle import bitlinear_oracle as O
+    x = d["x"][rows]
+    ops = 0
+    q4, xs4 = O.quant_act(x, O.MODE_INT4)
+    f4, xsf = O.quant_act(x, O.MODE_FP4)
+    for wt in (qkv_wt, gu_wt):
+        n_all = wt[0].shape[1]
+        w = n_all if width is None else width
+        Wt, g, e = _window(wt, (col0 * w) % n_all if width else 0, w)
+        O.bitlinear_int(q4, xs4, Wt, g, e)
+        O.bitlinear_fp4(f4, xsf, Wt, g, e)
+        ops += 2 * 2 * len(rows) * Wt.shape[0] * Wt.shape[1]
+    return ops
+
+
+def oracle_weights(d):
+    from oracle import bitlinear_oracle as O
+    qkv_p, gu_p = d["projs"]
+    return (O.ternarize(qkv_p.W, qkv_p.group_ends) + (qkv_p.group_ends,),
+            O.ternarize(gu_p.W, gu_p.group_ends) + (gu_p.group_ends,))
+
+
+def blas_threads():
+    try:
+        import threadpoolctl
+        info = threadpoolctl.threadpool_info()
+        n = [i.get("num_threads") for i in info if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def cpu_baseline(d, budget_s=12.0, block=64):
+    qkv_wt, gu_wt = oracle_weights(d)
+    ops, t, rows_done = 0.0, 0.0, 0
+    while t < budget_s and rows_done < M_TOK:
+        rows = np.arange(rows_done, min(M_TOK, rows_done + block))
+        t0 = time.perf_counter()
+        ops += oracle_sample(d, qkv_wt, gu_wt, rows)
+        t += time.perf_counter() - t0
+        rows_done += len(rows)
+    return {"value": round(ops / t / 1e12, 6), "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"first {rows_done} of {M_TOK} token rows through both variants "
+                      f"({t:.1f} s of CPU time; weight ternarisation untimed)"}
+
+
+def bench_reference(args, ws, rank):
+    """The oracle on host cores, as it stands, in the same metric."""
+    if rank != 0:
+        return None
+    import workloads as W
+    d = W.input_projection_prefill(seed=args.seed)
+    qkv_wt, gu_wt = oracle_weights(d)
+    block, width = 8, 512
+    for i in range(args.warmup):
+        s0 = (i * block) % M_TOK
+        oracle_sample(d, qkv_wt, gu_wt, np.arange(s0, s0 + block), i, width)
+    ops = 0.0
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        s0 = (i * block) % M_TOK
+        ops += oracle_sample(d, qkv_wt, gu_wt, np.arange(s0, s0 + block), i, width)
+    t = time.perf_counter() - t0
+    value = ops / t / 1e12
+    sample = (f"each step: {block} of the {M_TOK} token rows through both variants against a "
+              f"{width}-column window of each projection (rotating rows and windows)")
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TOPS",
+            "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t * 1e3 / args.steps, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (oracle)", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "tokens": M_TOK, "d_model": D},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TOPS", "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": "TOPS", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+# ------------------------------------------------------------ breakdown
+def _dev_bf16(torch, bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def breakdown(ctx, args):
+    """The other workloads of the path, each timed the same way (rotating
+    replicas larger than L2, CUDA graphs, per-launch events)."""
+    d, qkv, gu, reps, B, torch, dev, stream = ctx
+    import workloads as W
+    peaks, src = load_peaks()
+    hbm, int8_peak = peaks["hbm_gbs"], RATIO_INT8 * peaks["bf16_tflops"]
+    steps, warm = max(24, min(args.steps, 200)), 5
+    out = {"peaks": f"{src}: HBM {hbm} GB/s, int8 {int8_peak:.0f} TOPS (2 x bf16 burst)"}
+    mb = 1e6
+
+    # -- o_proj: top-k 50% + INT8, then the s8 GEMM 4096 x 4096 x 4096
+    o = W.o_proj_sparse()
+    Wp, g = B.ternarize_pack(o["proj"].W, (4096,))
+    M, K, N = 4096, 4096, 4096
+    bufs = []
+    for _ in range(3):
+        bufs.append(dict(x=_dev_bf16(torch, o["x"], dev), Wp=torch.from_numpy(Wp).to(dev),
+                         g=torch.from_numpy(g).to(dev), q=torch.empty((M, K), dtype=torch.int8, device=dev),
+                         xs=torch.empty(M, dtype=torch.float32, device=dev),
+                         y=torch.empty((M, N), dtype=torch.bfloat16, device=dev)))
+
+    def o_step(ev, b):
+        if ev: ev["topk"][0].record()
+        B.topk_sparsify_i8(b["x"], out=b["q"], xs=b["xs"])
+        if ev: ev["topk"][1].record(); ev["gemm"][0].record()
+        B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
+        if ev: ev["gemm"][1].record()
+    gs, es = graph_set(torch, stream, [(lambda ev, b=b: o_step(ev, b)) for b in bufs], ("topk", "gemm"), 8)
+    ms, k, _ = run_graphs(torch, stream, gs, es, ("topk", "gemm"), steps, warm)
+    ops = 2 * M * K * N
+    tb = M * K * 2 + M * K + M * 4
+    out["o_proj_topk_w2a8_4096x4096x4096"] = {
+        "step_us": round(ms / steps * 1e3, 2),
+        "gemm_us": round(k["gemm"] * 1e3, 2), "gemm_TOPS": round(ops / k["gemm"] / 1e9, 1),
+        "gemm_frac_int8": round(ops / k["gemm"] / 1e9 / int8_peak, 4),
+        "topk_us": round(k["topk"] * 1e3, 2), "topk_GBps": round(tb / k["topk"] / 1e6, 1),
+        "topk_frac_hbm": round(tb / k["topk"] / 1e6 / hbm, 4)}
+    del gs, es, bufs
+
+    # -- down_proj: ReLU^2 gate + INT8, then the s8 GEMM 4096 x 11008 x 4096
+    dn = W.down_proj_relu2()
+    Wp, g = B.ternarize_pack(dn["proj"].W, (4096,))
+    M, K, N = 4096, 11008, 4096
+    b = dict(gate=_dev_bf16(torch, dn["gate"], dev), up=_dev_bf16(torch, dn["up"], dev),
+             Wp=torch.from_numpy(Wp).to(dev), g=torch.from_numpy(g).to(dev),
+             q=torch.empty((M, K), dtype=torch.int8, device=dev),
+             xs=torch.empty(M, dtype=torch.float32, device=dev),
+             y=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
+    del dn
+
+    def d_step(ev):
+        if ev: ev["quant"][0].record()
+        B.quant_act(b["gate"], B.MODE_INT8, up=b["up"], out=b["q"], xs=b["xs"])
+        if ev: ev["quant"][1].record(); ev["gemm"][0].record()
+        B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
+        if ev: ev["gemm"][1].record()
+    gs, es = graph_set(torch, stream, [d_step], ("quant", "gemm"), 24)
+    ms, k, _ = run_graphs(torch, stream, gs, es, ("quant", "gemm"), steps, warm)
+    ops = 2 * M * K * N
+    qb = 2 * M * K * 2 + M * K + M * 4
+    zero_codes = float((b["q"] == 0).float().mean().item())
+    out["down_proj_relu2_w2a8_4096x11008x4096"] = {
+        "step_us": round(ms / steps * 1e3, 2),
+        "gemm_us": round(k["gemm"] * 1e3, 2), "gemm_TOPS": round(ops / k["gemm"] / 1e9, 1),
+        "gemm_frac_int8": round(ops / k["gemm"] / 1e9 / int8_peak, 4),
+        "relu2_quant_us": round(k["quant"] * 1e3, 2), "relu2_quant_GBps": round(qb / k["quant"] / 1e6, 1),
+        "relu2_quant_frac_hbm": round(qb / k["quant"] / 1e6 / hbm, 4),
+        "zero_code_fraction": round(zero_codes, 4)}
+    del gs, es, b
+
+    # -- decode: one LLaMA-7B-shaped layer at batch 1 / 8 / 64
+    lay = W.decode_layer(batch=64, make_kv=False)
+    packed = [B.ternarize_pack(p.W, p.group_ends) for p in lay["projs"]]
+    shapes = [(p.name, p.K, p.N) for p in lay["projs"]]
+    wbytes = sum(p.K * p.N // 4 for p in lay["projs"])
+    R = 6
+    wdev = [[(torch.from_numpy(wp).to(dev), torch.from_numpy(gm).to(dev)) for wp, gm in packed]
+            for _ in range(R)]
+    dec = {}
+    names = tuple(n for n, _, _ in shapes)
+    for batch in (1, 8, 64):
+        x = _dev_bf16(torch, lay["x"][:batch], dev)
+        xo = _dev_bf16(torch, lay["xo"][:batch], dev)
+        ga = _dev_bf16(torch, lay["gate"][:batch], dev)
+        up = _dev_bf16(torch, lay["up"][:batch], dev)
+        ys = {n: torch.empty((batch, N), dtype=torch.bfloat16, device=dev) for n, _, N in shapes}
+
+        def l_step(ev, r):
+            ws_ = wdev[r]
+            q, xs = B.quant_act(x, B.MODE_INT4)
+            for i, n in enumerate(("q", "k", "v")):
+                if ev: ev[n][0].record()
+                B.gemv_w2(q, xs, ws_[i][0], ws_[i][1], (4096,), y=ys[n])
+                if ev: ev[n][1].record()
+            qo, xso, _ = B.topk_sparsify_i8(xo)
+            if ev: ev["o"][0].record()
+            B.gemv_w2(qo, xso, ws_[3][0], ws_[3][1], (4096,), y=ys["o"])
+            if ev: ev["o"][1].record()
+            for i, n in ((4, "gate"), (5, "up")):
+                if ev: ev[n][0].record()
+                B.gemv_w2(q, xs, ws_[i][0], ws_[i][1], (11008,), y=ys[n])
+                if ev: ev[n][1].record()
+            qd, xsd = B.quant_act(ga, B.MODE_INT8, up=up)
+            if ev: ev["down"][0].record()
+            B.gemv_w2(qd, xsd, ws_[6][0], ws_[6][1], (4096,), y=ys["down"])
+            if ev: ev["down"][1].record()
+        gs, es = graph_set(torch, stream, [(lambda ev, r=r: l_step(ev, r)) for r in range(R)], names, 4)
+        ms, k, _ = run_graphs(torch, stream, gs, es, names, steps, warm)
+        gemv_ms = sum(k.values())
+        per = {n: {"us": round(k[n] * 1e3, 2),
+                   "GBps": round(K_ * N_ // 4 / k[n] / 1e6, 1)} for n, K_, N_ in shapes}
+        dec[f"batch{batch}"] = {
+            "layer_step_us": round(ms / steps * 1e3, 2),
+            "gemv_sum_us": round(gemv_ms * 1e3, 2),
+            "weight_GBps": round(wbytes / gemv_ms / 1e6, 1),
+            "weight_frac_hbm": round(wbytes / gemv_ms / 1e6 / hbm, 4),
+            "layer_weight_GBps_incl_quantisers": round(wbytes / (ms / steps) / 1e6, 1),
+            "per_projection": per}
+        del gs, es
+    out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=11, **dec)
+    del wdev
+
+    # -- KV cache: K and V [4096 x 32 x 128] -> 3-bit codes, bos at 4 bits
+    kvd = W.decode_layer(batch=1, make_weights=False)
+    keep = torch.tensor([0], dtype=torch.int32, device=dev)
+    kvs = [(_dev_bf16(torch, kvd["k_cache"], dev), _dev_bf16(torch, kvd["v_cache"], dev)) for _ in range(4)]
+    T, H, Dh = kvd["k_cache"].shape
+    o3 = [torch.empty((T, H, 3 * Dh // 8), dtype=torch.uint8, device=dev) for _ in range(2)]
+    o4 = [torch.empty((1, H, Dh // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
+    sc = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(2)]
+
+    def kv_step(ev, r):
+        if ev: ev["kv"][0].record()
+        for j in range(2):
+            B.kv_quant_3bit(kvs[r][j], keep, codes3=o3[j], codes4=o4[j], scale=sc[j])
+        if ev: ev["kv"][1].record()
+    gs, es = graph_set(torch, stream, [(lambda ev, r=r: kv_step(ev, r)) for r in range(4)], ("kv",), 6)
+    ms, k, _ = run_graphs(torch, stream, gs, es, ("kv",), steps, warm)
+    kb = 2 * (T * H * Dh * 2 + T * H * 3 * Dh // 8 + T * H * 4 + H * Dh // 2)
+    out["kv_quant_3bit_2x4096x32x128"] = {"us": round(k["kv"] * 1e3, 2),
+                                         "GBps": round(kb / k["kv"] / 1e6, 1),
+                                         "frac_hbm": round(kb / k["kv"] / 1e6 / hbm, 4)}
+    del gs, es
+    B.check_status(stream=stream)
+    return out
+
+
+def main():
+    args = parse()
+    ws, rank, local = dist_init()
+    if args.impl == "reference":
+        out = bench_reference(args, ws, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    out, ctx = bench_ours(args, ws, rank, local)
+    if not args.no_e2e:
+        out["e2e"] = bench_e2e(args, ctx, ws)
+    if rank == 0 and ws == 1 and not args.no_breakdown:
+        out["breakdown"] = breakdown(ctx, args)
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(ctx[0])
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

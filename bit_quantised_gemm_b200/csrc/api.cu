@@ -45,6 +45,7 @@ int check_gemm(const char* fn, const void* xq, const void* xs, const uint8_t* Wp
   if (N % 16 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: N=%lld must be a multiple of 16", fn, (long long)N);
   if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 24))
     return fail(BITLINEAR_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
+  if (M == 0) return BITLINEAR_OK;  // empty call: pointers may be null, nothing is launched
   if (!xq || !Wp || !y) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: null operand pointer", fn);
   if (!aligned16(xq) || !aligned16(Wp) || !aligned16(y))
     return fail(BITLINEAR_ERR_ALIGNMENT, "%s: operands must be 16-byte aligned", fn);
@@ -106,9 +107,12 @@ EncodeTiledFn get_encode_tiled() {
 }
 
 int num_sms() {
+  static int cache[64] = {0};
   int dev = 0, n = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 1;
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
   if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) return 1;
+  if (dev >= 0 && dev < 64) cache[dev] = n;
   return n;
 }
 
@@ -143,7 +147,6 @@ int bitlinear_ternarize_pack(const float* W, int64_t K, int64_t N, const int64_t
   }
   if (prev != N) return fail(BITLINEAR_ERR_INVALID_ARG, "ternarize_pack: last group end must equal N");
 
-  std::vector<int8_t> col_code(static_cast<size_t>(N));  // reused per row
   std::vector<float> g(G);
   int64_t start = 0;
   for (int gi = 0; gi < G; ++gi) {
@@ -175,7 +178,6 @@ int bitlinear_ternarize_pack(const float* W, int64_t K, int64_t N, const int64_t
     }
     start = end;
   }
-  (void)col_code;
   return ok();
 }
 
@@ -187,6 +189,7 @@ int bitlinear_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, int64_
   if (K > 49152) return fail(BITLINEAR_ERR_UNSUPPORTED, "quant_act: K above 49152");
   if (M > 0x7FFFFFFF) return fail(BITLINEAR_ERR_UNSUPPORTED, "quant_act: too many rows");
   if (ldx < K || ldx % 8 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "quant_act: ldx must be >= K and a multiple of 8");
+  if (M == 0) return ok();
   if (!x || !q_out || !xs_out) return fail(BITLINEAR_ERR_INVALID_ARG, "quant_act: null pointer");
   if (!aligned16(x) || (up && !aligned16(up)) || !aligned16(q_out))
     return fail(BITLINEAR_ERR_ALIGNMENT, "quant_act: pointers must be 16-byte aligned");
@@ -203,6 +206,7 @@ int bitlinear_topk_sparsify_i8(const uint16_t* x, int64_t M, int64_t K, int64_t 
   if (M > 0x7FFFFFFF) return fail(BITLINEAR_ERR_UNSUPPORTED, "topk: too many rows");
   if (k < 0) return fail(BITLINEAR_ERR_INVALID_ARG, "topk: k must be >= 0");
   if (ldx < K || ldx % 8 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "topk: ldx must be >= K and a multiple of 8");
+  if (M == 0) return ok();
   if (!x || !q_out || !xs_out) return fail(BITLINEAR_ERR_INVALID_ARG, "topk: null pointer");
   if (!aligned16(x) || !aligned16(q_out)) return fail(BITLINEAR_ERR_ALIGNMENT, "topk: pointers must be 16-byte aligned");
   if (k == 0) k = (K + 1) / 2;
@@ -217,10 +221,10 @@ static int gemm_common(const char* fn, const void* xq, const float* xs, const ui
                        int64_t K, void* out, int64_t ldo, int out_mode, int* dev_status, bool fp4,
                        bitlinear_stream_t stream) {
   blt::GemmArgs a{};
+  if (fp4 && K % 128 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: K must be a multiple of 128", fn);
   const int rc = check_gemm(fn, xq, xs, Wp, gamma, group_ends, G, M, N, K, out, ldo,
                             out_mode == blt::kOutBf16, &a);
   if (rc != BITLINEAR_OK) return rc;
-  if (fp4 && K % 128 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: K must be a multiple of 128", fn);
   if (M == 0) return ok();
   a.out = out;
   a.ldo = ldo;
@@ -269,10 +273,10 @@ int bitlinear_gemv_w2(const int8_t* xq, const float* xs, const uint8_t* Wp, cons
                       const int64_t* group_ends, int G, int64_t M, int64_t N, int64_t K,
                       uint16_t* y, int64_t ldy, int* dev_status, bitlinear_stream_t stream) {
   blt::GemmArgs a{};
-  const int rc = check_gemm("gemv_w2", xq, xs, Wp, gamma, group_ends, G, M, N, K, y, ldy, true, &a);
-  if (rc != BITLINEAR_OK) return rc;
   if (M > 64) return fail(BITLINEAR_ERR_INVALID_ARG, "gemv_w2: M=%lld above 64 (use a GEMM)", (long long)M);
   if (K % 128 != 0 || N % 128 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "gemv_w2: K and N must be multiples of 128");
+  const int rc = check_gemm("gemv_w2", xq, xs, Wp, gamma, group_ends, G, M, N, K, y, ldy, true, &a);
+  if (rc != BITLINEAR_OK) return rc;
   if (M == 0) return ok();
   a.out = y;
   a.ldo = ldy;
@@ -290,6 +294,7 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
   if (D != 64 && D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: D must be 64, 128 or 256");
   if (n_keep4 < 0 || n_keep4 > T || (n_keep4 > 0 && (!keep4_pos || !codes4)))
     return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: bad 4-bit token list");
+  if (T == 0) return ok();
   if (!kv || !codes3 || !scale) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: null pointer");
   if (!aligned16(kv) || !aligned16(codes3) || (codes4 && !aligned16(codes4)))
     return fail(BITLINEAR_ERR_ALIGNMENT, "kv_quant_3bit: pointers must be 16-byte aligned");

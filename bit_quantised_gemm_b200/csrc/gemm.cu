@@ -316,8 +316,12 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.timeout_ns = a.timeout_ns;
 
   auto kern = fp4 ? bitlinear_gemm_kernel<true> : bitlinear_gemm_kernel<false>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  static bool attr_set[2] = {false, false};  // once per process (not during graph capture)
+  if (!attr_set[fp4 ? 1 : 0]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set[fp4 ? 1 : 0] = true;
+  }
   const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
   kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmW, p);
   return cudaGetLastError();

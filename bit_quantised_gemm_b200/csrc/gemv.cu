@@ -288,9 +288,13 @@ cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why) {
       return cudaErrorInvalidValue;
     }
   }
-  cudaError_t e = cudaFuncSetAttribute(bitlinear_gemv_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-  if (e != cudaSuccess) return e;
+  static bool attr_set = false;  // once per process (not during graph capture)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(bitlinear_gemv_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(tiles * c));
   cfg.blockDim = dim3(THREADS);

@@ -142,10 +142,12 @@ static cudaError_t launch_quant_t(const uint16_t* x, const uint16_t* up, int64_t
                                   int64_t ldx, void* q, float* xs, cudaStream_t s) {
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
   auto kern = quant_act_kernel<MODE, RELU2>;
-  if (smem > 48 * 1024) {
+  static int attr_bytes = 48 * 1024;  // raised once, monotonically (outside graph capture in practice)
+  if (static_cast<int>(smem) > attr_bytes) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
+    attr_bytes = static_cast<int>(smem);
   }
   kern<<<static_cast<unsigned>(M), kQuantThreads, smem, s>>>(x, up, K, ldx, q, xs);
   return cudaGetLastError();

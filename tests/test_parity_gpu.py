@@ -73,7 +73,7 @@ def test_fp4_rounding_midpoints():
     vals = []
     for m in mids:
         b = O.f32_to_bf16(np.float32(m))
-        vals += [m, float(O.bf16_to_f32(b + 1)), float(O.bf16_to_f32(b - 1))]
+        vals += [m, float(O.bf16_to_f32(b + 1)[()]), float(O.bf16_to_f32(b - 1)[()])]
     vals += [0.0, -0.0, 0.1, -0.1, 6.0, 4.0, 3.0]
     vals += [-v for v in vals]
     row = np.array(vals + [0.0] * (-len(vals) % 16), np.float32)
