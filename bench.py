@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--section", default=None,
+                    help="run only one breakdown section (o_proj, down_proj, decode, kv), e.g. "
+                         "to profile its kernels; prints that section's JSON")
     return ap.parse_args()
 
 
@@ -477,18 +480,28 @@ def _dev_bf16(torch, bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
 
-def breakdown(ctx, args):
+SECTIONS = ("o_proj", "down_proj", "decode", "kv")
+
+
+def breakdown(ctx, args, sections=SECTIONS):
     """The other workloads of the path, each timed the same way (rotating
     replicas larger than L2, CUDA graphs, per-launch events)."""
-    d, qkv, gu, reps, B, torch, dev, stream = ctx
-    import workloads as W
+    B, torch, dev, stream = ctx[4], ctx[5], ctx[6], ctx[7]
     peaks, src = load_peaks()
-    hbm, int8_peak = peaks["hbm_gbs"], RATIO_INT8 * peaks["bf16_tflops"]
-    steps, warm = max(24, min(args.steps, 200)), 5
-    out = {"peaks": f"{src}: HBM {hbm} GB/s, int8 {int8_peak:.0f} TOPS (2 x bf16 burst)"}
-    mb = 1e6
+    out = {"peaks": f"{src}: HBM {peaks['hbm_gbs']} GB/s, int8 {RATIO_INT8 * peaks['bf16_tflops']:.0f} "
+                    "TOPS (2 x bf16 burst)"}
+    steps, warm = max(24, min(args.steps, 200)), min(5, args.warmup)
+    for name in sections:
+        out.update(globals()["section_" + name](B, torch, dev, stream, peaks, steps, warm))
+    B.check_status(stream=stream)
+    return out
 
-    # -- o_proj: top-k 50% + INT8, then the s8 GEMM 4096 x 4096 x 4096
+
+def section_o_proj(B, torch, dev, stream, peaks, steps, warm):
+    """o_proj: top-k 50% + INT8, then the s8 GEMM 4096 x 4096 x 4096."""
+    import workloads as W
+    hbm, int8_peak = peaks["hbm_gbs"], RATIO_INT8 * peaks["bf16_tflops"]
+    out = {}
     o = W.o_proj_sparse()
     Wp, g = B.ternarize_pack(o["proj"].W, (4096,))
     M, K, N = 4096, 4096, 4096
@@ -515,9 +528,14 @@ def breakdown(ctx, args):
         "gemm_frac_int8": round(ops / k["gemm"] / 1e9 / int8_peak, 4),
         "topk_us": round(k["topk"] * 1e3, 2), "topk_GBps": round(tb / k["topk"] / 1e6, 1),
         "topk_frac_hbm": round(tb / k["topk"] / 1e6 / hbm, 4)}
-    del gs, es, bufs
+    return out
 
-    # -- down_proj: ReLU^2 gate + INT8, then the s8 GEMM 4096 x 11008 x 4096
+
+def section_down_proj(B, torch, dev, stream, peaks, steps, warm):
+    """down_proj: ReLU^2 gate + INT8, then the s8 GEMM 4096 x 11008 x 4096."""
+    import workloads as W
+    hbm, int8_peak = peaks["hbm_gbs"], RATIO_INT8 * peaks["bf16_tflops"]
+    out = {}
     dn = W.down_proj_relu2()
     Wp, g = B.ternarize_pack(dn["proj"].W, (4096,))
     M, K, N = 4096, 11008, 4096
@@ -546,49 +564,68 @@ def breakdown(ctx, args):
         "relu2_quant_us": round(k["quant"] * 1e3, 2), "relu2_quant_GBps": round(qb / k["quant"] / 1e6, 1),
         "relu2_quant_frac_hbm": round(qb / k["quant"] / 1e6 / hbm, 4),
         "zero_code_fraction": round(zero_codes, 4)}
-    del gs, es, b
+    return out
 
-    # -- decode: one LLaMA-7B-shaped layer at batch 1 / 8 / 64
+
+def section_decode(B, torch, dev, stream, peaks, steps, warm):
+    """Decode: one LLaMA-7B-shaped layer at batch 1 / 8 / 64 (weight GB/s).
+
+    The projections that share an input run as one launch with per-group
+    scales (q|k|v: N = 12288, 3 groups; gate|up: N = 22016, 2 groups), then
+    o (4096) and down (11008 -> 4096): four GEMV launches per layer."""
+    import workloads as W
+    hbm = peaks["hbm_gbs"]
+    out = {}
     lay = W.decode_layer(batch=64, make_kv=False)
-    packed = [B.ternarize_pack(p.W, p.group_ends) for p in lay["projs"]]
-    shapes = [(p.name, p.K, p.N) for p in lay["projs"]]
-    wbytes = sum(p.K * p.N // 4 for p in lay["projs"])
-    R = 6
-    wdev = [[(torch.from_numpy(wp).to(dev), torch.from_numpy(gm).to(dev)) for wp, gm in packed]
+    P = {p.name: p for p in lay["projs"]}
+    D, F = P["q"].K, P["gate"].N
+    fused = {
+        "qkv": (np.concatenate([P["q"].W, P["k"].W, P["v"].W], axis=1), (D, 2 * D, 3 * D)),
+        "o": (P["o"].W, (D,)),
+        "gate_up": (np.concatenate([P["gate"].W, P["up"].W], axis=1), (F, 2 * F)),
+        "down": (P["down"].W, (D,)),
+    }
+    packed = {k: B.ternarize_pack(w, ge) for k, (w, ge) in fused.items()}
+    shapes = {k: (w.shape[0], w.shape[1], ge) for k, (w, ge) in fused.items()}
+    del fused, lay["projs"]
+    wbytes = sum(K * N // 4 for K, N, _ in shapes.values())
+    R = 6  # weight replicas: 6 x 48 MB > 2 x L2
+    wdev = [{k: (torch.from_numpy(wp).to(dev), torch.from_numpy(gm).to(dev)) for k, (wp, gm) in packed.items()}
             for _ in range(R)]
+    names = tuple(shapes)
     dec = {}
-    names = tuple(n for n, _, _ in shapes)
     for batch in (1, 8, 64):
         x = _dev_bf16(torch, lay["x"][:batch], dev)
         xo = _dev_bf16(torch, lay["xo"][:batch], dev)
         ga = _dev_bf16(torch, lay["gate"][:batch], dev)
         up = _dev_bf16(torch, lay["up"][:batch], dev)
-        ys = {n: torch.empty((batch, N), dtype=torch.bfloat16, device=dev) for n, _, N in shapes}
+        ys = {k: torch.empty((batch, N), dtype=torch.bfloat16, device=dev) for k, (_, N, _) in shapes.items()}
+        q4 = torch.empty((batch, D), dtype=torch.int8, device=dev)
+        xs4 = torch.empty(batch, dtype=torch.float32, device=dev)
+        qo = torch.empty((batch, D), dtype=torch.int8, device=dev)
+        xso = torch.empty(batch, dtype=torch.float32, device=dev)
+        qd = torch.empty((batch, F), dtype=torch.int8, device=dev)
+        xsd = torch.empty(batch, dtype=torch.float32, device=dev)
+
+        def gemv(ev, name, xq, xs, wr):
+            if ev: ev[name][0].record()
+            B.gemv_w2(xq, xs, wr[name][0], wr[name][1], shapes[name][2], y=ys[name])
+            if ev: ev[name][1].record()
 
         def l_step(ev, r):
-            ws_ = wdev[r]
-            q, xs = B.quant_act(x, B.MODE_INT4)
-            for i, n in enumerate(("q", "k", "v")):
-                if ev: ev[n][0].record()
-                B.gemv_w2(q, xs, ws_[i][0], ws_[i][1], (4096,), y=ys[n])
-                if ev: ev[n][1].record()
-            qo, xso, _ = B.topk_sparsify_i8(xo)
-            if ev: ev["o"][0].record()
-            B.gemv_w2(qo, xso, ws_[3][0], ws_[3][1], (4096,), y=ys["o"])
-            if ev: ev["o"][1].record()
-            for i, n in ((4, "gate"), (5, "up")):
-                if ev: ev[n][0].record()
-                B.gemv_w2(q, xs, ws_[i][0], ws_[i][1], (11008,), y=ys[n])
-                if ev: ev[n][1].record()
-            qd, xsd = B.quant_act(ga, B.MODE_INT8, up=up)
-            if ev: ev["down"][0].record()
-            B.gemv_w2(qd, xsd, ws_[6][0], ws_[6][1], (4096,), y=ys["down"])
-            if ev: ev["down"][1].record()
+            wr = wdev[r]
+            B.quant_act(x, B.MODE_INT4, out=q4, xs=xs4)
+            gemv(ev, "qkv", q4, xs4, wr)
+            B.topk_sparsify_i8(xo, out=qo, xs=xso)
+            gemv(ev, "o", qo, xso, wr)
+            gemv(ev, "gate_up", q4, xs4, wr)
+            B.quant_act(ga, B.MODE_INT8, up=up, out=qd, xs=xsd)
+            gemv(ev, "down", qd, xsd, wr)
         gs, es = graph_set(torch, stream, [(lambda ev, r=r: l_step(ev, r)) for r in range(R)], names, 4)
         ms, k, _ = run_graphs(torch, stream, gs, es, names, steps, warm)
         gemv_ms = sum(k.values())
-        per = {n: {"us": round(k[n] * 1e3, 2),
-                   "GBps": round(K_ * N_ // 4 / k[n] / 1e6, 1)} for n, K_, N_ in shapes}
+        per = {n: {"us": round(k[n] * 1e3, 2), "GBps": round(K_ * N_ // 4 / k[n] / 1e6, 1)}
+               for n, (K_, N_, _) in shapes.items()}
         dec[f"batch{batch}"] = {
             "layer_step_us": round(ms / steps * 1e3, 2),
             "gemv_sum_us": round(gemv_ms * 1e3, 2),
@@ -597,10 +634,17 @@ def breakdown(ctx, args):
             "layer_weight_GBps_incl_quantisers": round(wbytes / (ms / steps) / 1e6, 1),
             "per_projection": per}
         del gs, es
-    out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=11, **dec)
-    del wdev
+    out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=7,
+                                       gemv_launches="qkv (fused, 3 groups), o, gate_up (fused, 2 groups), down",
+                                       **dec)
+    return out
 
-    # -- KV cache: K and V [4096 x 32 x 128] -> 3-bit codes, bos at 4 bits
+
+def section_kv(B, torch, dev, stream, peaks, steps, warm):
+    """KV cache: K and V [4096 x 32 x 128] -> 3-bit codes, bos at 4 bits."""
+    import workloads as W
+    hbm = peaks["hbm_gbs"]
+    out = {}
     kvd = W.decode_layer(batch=1, make_weights=False)
     keep = torch.tensor([0], dtype=torch.int32, device=dev)
     kvs = [(_dev_bf16(torch, kvd["k_cache"], dev), _dev_bf16(torch, kvd["v_cache"], dev)) for _ in range(4)]
@@ -620,14 +664,21 @@ def breakdown(ctx, args):
     out["kv_quant_3bit_2x4096x32x128"] = {"us": round(k["kv"] * 1e3, 2),
                                          "GBps": round(kb / k["kv"] / 1e6, 1),
                                          "frac_hbm": round(kb / k["kv"] / 1e6 / hbm, 4)}
-    del gs, es
-    B.check_status(stream=stream)
     return out
 
 
 def main():
     args = parse()
     ws, rank, local = dist_init()
+    if args.section:
+        import torch
+        import bit_quantised_gemm_b200 as B
+        torch.cuda.set_device(local)
+        B.lib()
+        stream = torch.cuda.Stream(device=f"cuda:{local}")
+        ctx = (None, None, None, None, B, torch, f"cuda:{local}", stream)
+        print(json.dumps(breakdown(ctx, args, (args.section,))), flush=True)
+        return
     if args.impl == "reference":
         out = bench_reference(args, ws, rank)
         if out is not None:

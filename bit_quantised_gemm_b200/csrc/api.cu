@@ -43,7 +43,7 @@ int check_gemm(const char* fn, const void* xq, const void* xs, const uint8_t* Wp
   if (M < 0 || N <= 0 || K <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: bad sizes M=%lld N=%lld K=%lld", fn, (long long)M, (long long)N, (long long)K);
   if (K % 64 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: K=%lld must be a multiple of 64", fn, (long long)K);
   if (N % 16 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: N=%lld must be a multiple of 16", fn, (long long)N);
-  if (M > (1LL << 30) || N > (1LL << 30) || K > (1LL << 24))
+  if (M > (1LL << 30) || N > (1LL << 30) || K > 32768)
     return fail(BITLINEAR_ERR_UNSUPPORTED, "%s: sizes beyond the supported range", fn);
   if (M == 0) return BITLINEAR_OK;  // empty call: pointers may be null, nothing is launched
   if (!xq || !Wp || !y) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: null operand pointer", fn);

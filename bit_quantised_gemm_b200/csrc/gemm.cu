@@ -2,19 +2,25 @@
 //
 //   acc[m, n] = sum_k a[m, k] * w[k, n],  a = int8 codes (kind::i8, s32 acc)
 //                                          or e2m1 codes (kind::f8f6f4, f32 acc)
-//   y[m, n]   = bf16(acc * xs[m] * gamma[group(n)])   (or the raw acc)
+//   y[m, n]   = bf16(acc * (xs[m] * gamma[group(n)]))   (or the raw acc)
 //
-// Persistent, warp-specialised kernel, one 128 x 256 output tile at a time:
-//   warp 0      TMA producer: activation tile (128 x 128 B, 128-byte swizzle)
-//               and packed-weight tile (256 rows x 32 B) into a 5-stage ring
-//   warp 1      TMEM allocator and single-thread MMA issuer (4 MMAs of
-//               K = 32 per 128-deep k-block, accumulator in TMEM)
-//   warps 4-7   epilogue: tcgen05.ld of the accumulator (lane = row), scale,
-//               bf16 pack, 16-byte global stores; TMEM holds two accumulators
-//               so the epilogue of tile i overlaps the mainloop of tile i+1
+// Persistent, warp-specialised kernel. In the CTA-pair form (two CTAs of a
+// cluster on one TPC, tcgen05 cta_group::2) a pair owns a 256-token x
+// 256-output tile: each CTA loads its own 128 token rows of activations and
+// unpacks its own 128 weight rows, and one MMA of M = 256 reads both CTAs'
+// shared memory, so each SM stages half of the unpacked weights (the
+// single-CTA form stages all 256 rows and is used for M <= 128).
+//   warp 0      TMA producer: activation tile (128 rows x 128 B, 128-byte
+//               swizzle) and packed-weight tile (128 or 256 rows x 32 B) into
+//               one ring slot
+//   warp 1      TMEM allocator; in the even CTA the single-thread MMA issuer
+//               (4 MMAs of K = 32 per 128-deep k-block, accumulator in TMEM)
+//   warps 4-7   epilogue: tcgen05.ld (lane = token row), scale, bf16 pack,
+//               16-byte global stores; two TMEM accumulators so the epilogue
+//               of one tile overlaps the mainloop of the next
 //   warps 8-15  unpack: 2-bit weights -> int8 / padded e2m1 K-major tiles in
-//               the 128-byte swizzled layout the MMA descriptors describe
-//               (3-stage ring), then fence.proxy.async and an mbarrier arrive
+//               the swizzled layout the MMA descriptors describe, then
+//               fence.proxy.async and an mbarrier arrive (on the even CTA)
 // All waits are bounded (see ptx.cuh); a timeout sets a status bit and the
 // CTA unwinds, releasing TMEM.
 #include "common.cuh"
@@ -24,21 +30,36 @@
 namespace blt {
 namespace gemm {
 
-constexpr int BM = 128, BN = 256, BK = 128;  // BK counted in elements
-constexpr int S_TMA = 5, S_B = 3;
-constexpr int A_BYTES = BM * 128;            // one 128-byte row per token
-constexpr int WP_BYTES = BN * (BK / 4);      // 32 bytes of packed weights per row
-constexpr int B_BYTES = BN * 128;
-constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + S_TMA * A_BYTES;
-constexpr int OFF_WP = OFF_B + S_B * B_BYTES;
-constexpr int OFF_BAR = OFF_WP + S_TMA * WP_BYTES;
-constexpr int N_BARS = 2 * S_TMA + 2 * S_B + 2 * 2 + 1;
-constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+constexpr int BM = 128;            // token rows per CTA
+constexpr int BN = 256;            // output columns per tile
+constexpr int SUB = BM * 128;      // one 128-deep K chunk of activations: 128 rows x 128 B
 constexpr int THREADS = 512;
 constexpr int TMEM_COLS = 512;
-static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// A TMA instruction costs the issuing thread a few hundred ns whatever its
+// size, so the CTA-pair form moves 256-deep k-blocks (32 KB of activations in
+// one 3-D box) and splits the activation and weight loads over two warps.
+template <bool PAIR>
+struct Layout {
+  static constexpr int BK = PAIR ? 256 : 128;       // k-block depth in elements
+  static constexpr int KSUB = BK / 128;             // 128-deep swizzled chunks per k-block
+  static constexpr int S_TMA = PAIR ? 4 : 5;        // activation ring
+  static constexpr int S_W = PAIR ? 3 : 4;          // packed-weight ring
+  static constexpr int S_B = PAIR ? 2 : 3;          // unpacked-weight ring
+  static constexpr int BROWS = PAIR ? BN / 2 : BN;  // weight rows staged per CTA
+  static constexpr int A_BYTES = KSUB * SUB;
+  static constexpr int WP_BYTES = BROWS * (BK / 4);
+  static constexpr int B_BYTES = BROWS * BK;
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + S_TMA * A_BYTES;
+  static constexpr int OFF_WP = OFF_B + S_B * B_BYTES;
+  static constexpr int OFF_STG = OFF_WP + S_W * WP_BYTES;  // epilogue staging, 2 KB per warp
+  static constexpr int OFF_BAR = OFF_STG + 4 * 2048;
+  static constexpr int N_BARS = 2 * S_TMA + 2 * S_W + 2 * S_B + 2 * 2 + 1;
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
 
 struct Params {
   int M, N, K, num_kb, tiles_m, num_tiles;
@@ -53,37 +74,47 @@ struct Params {
   uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ float gamma_of(const Params& p, int n) {
+__device__ __forceinline__ int group_of(const Params& p, int n) {
   int g = 0;
 #pragma unroll
   for (int i = 0; i < 7; ++i) g += (i < p.G - 1 && n >= p.group_end[i]) ? 1 : 0;
-  return __ldg(p.gamma + g);
+  return g;
 }
 
-template <bool FP4>
+template <bool FP4, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmW, const Params p) {
+  using L = Layout<PAIR>;
+  constexpr int S_TMA = L::S_TMA, S_W = L::S_W, S_B = L::S_B, BK = L::BK, A_BYTES = L::A_BYTES;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  uint64_t* full = bars;                    // TMA landed     [S_TMA]
-  uint64_t* empty = full + S_TMA;           // MMA done with A/Wp slot [S_TMA]
-  uint64_t* bfull = empty + S_TMA;          // unpacked B ready [S_B]
-  uint64_t* bempty = bfull + S_B;           // MMA done with B slot [S_B]
-  uint64_t* tfull = bempty + S_B;           // accumulator ready [2]
-  uint64_t* tempty = tfull + 2;             // accumulator drained [2]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::OFF_BAR);
+  uint64_t* afull = bars;                   // activations landed (even CTA: both CTAs' bytes)
+  uint64_t* empty = afull + S_TMA;          // MMA done with activation slot (both CTAs)
+  uint64_t* wfull = empty + S_TMA;          // this CTA's packed weights landed
+  uint64_t* wempty = wfull + S_W;           // unpack done reading packed-weight slot
+  uint64_t* bfull = wempty + S_W;           // unpacked B ready (even CTA: both CTAs' warps)
+  uint64_t* bempty = bfull + S_B;           // MMA done with B slot (both CTAs)
+  uint64_t* tfull = bempty + S_B;           // accumulator ready (both CTAs)
+  uint64_t* tempty = tfull + 2;             // accumulator drained (even CTA: both epilogues)
   uint64_t* mma_done = tempty + 2;          // all MMAs retired (teardown)
-  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
-  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const bool leader = rank == 0;
+  const int cta_slot = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int cta_stride = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
+  constexpr int TILE_M = PAIR ? 2 * BM : BM;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < S_TMA; ++i) { mbar_init(&full[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < S_B; ++i) { mbar_init(&bfull[i], 256); mbar_init(&bempty[i], 1); }
-    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], 128); }
+    for (int i = 0; i < S_TMA; ++i) { mbar_init(&afull[i], 1); mbar_init(&empty[i], 1); }
+    for (int i = 0; i < S_W; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], 8); }
+    for (int i = 0; i < S_B; ++i) { mbar_init(&bfull[i], PAIR ? 16 : 8); mbar_init(&bempty[i], 1); }
+    for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], PAIR ? 8 : 4); }
     mbar_init(mma_done, 1);
     *s_abort = 0;
     fence_mbar_init();
@@ -91,92 +122,135 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     prefetch_tensormap(&tmW);
   }
   if (warp == 1) {
-    tmem_alloc(s_tmem, TMEM_COLS);
-    tmem_relinquish();
+    if (PAIR) { tmem_alloc_pair(s_tmem, TMEM_COLS); tmem_relinquish_pair(); }
+    else      { tmem_alloc(s_tmem, TMEM_COLS); tmem_relinquish(); }
   }
   __syncthreads();
+  if (PAIR) cluster_sync();  // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
 
-  const uint32_t sA = smem_u32(smem + OFF_A);
-  const uint32_t sB = smem_u32(smem + OFF_B);
-  const uint32_t sW = smem_u32(smem + OFF_WP);
+  const uint32_t sA = smem_u32(smem + L::OFF_A);
+  const uint32_t sB = smem_u32(smem + L::OFF_B);
+  const uint32_t sW = smem_u32(smem + L::OFF_WP);
   const uint64_t tmo = p.timeout_ns;
-
+  // barrier addresses in the even CTA of the pair (or this CTA)
+  auto lead = [&](uint64_t* bar) -> uint32_t {
+    return PAIR ? map_shared_rank(smem_u32(bar), 0) : smem_u32(bar);
+  };
   auto fail = [&]() {
     *s_abort = 1;
     report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
   };
+  constexpr uint32_t A_TX = FP4 ? L::A_BYTES / 2 : L::A_BYTES;  // global bytes (packed e2m1 = half)
 
-  if (warp == 0) {
-    // ------------------------------------------------------ TMA producer
+  if (warp == 0 || warp == 2) {
+    // ----------------------------------------- TMA producers (A: warp 0, W: warp 2)
     if (lane == 0) {
+      const bool act = warp == 0;
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
-        const int m0 = (tile % p.tiles_m) * BM, n0 = (tile / p.tiles_m) * BN;
+      for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride) {
+        const int m0 = (tile % p.tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+        const int n0 = (tile / p.tiles_m) * BN + static_cast<int>(rank) * L::BROWS;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-          const uint32_t s = it % S_TMA, ph = (it / S_TMA) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, tmo, s_abort)) { fail(); ok = false; break; }
-          // transaction bytes count global bytes: packed e2m1 is half its smem footprint
-          mbar_arrive_expect_tx(&full[s], (FP4 ? A_BYTES / 2 : A_BYTES) + WP_BYTES);
-          tma_load_2d(smem + OFF_A + s * A_BYTES, &tmA, &full[s], kb * BK, m0);
-          tma_load_2d(smem + OFF_WP + s * WP_BYTES, &tmW, &full[s], kb * (BK / 4), n0);
+          const int S = act ? S_TMA : S_W;
+          const uint32_t s = it % S, ph = (it / S) & 1;
+          if (!mbar_wait(act ? &empty[s] : &wempty[s], ph ^ 1, tmo, s_abort)) { fail(); ok = false; break; }
+          if (act) {
+            uint8_t* dst = smem + L::OFF_A + s * A_BYTES;
+            if (PAIR) {
+              if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
+              tma_load_3d_pair(dst, &tmA, lead(&afull[s]), 0, m0, kb * L::KSUB);
+            } else {
+              mbar_arrive_expect_tx(&afull[s], A_TX);
+              tma_load_2d(dst, &tmA, &afull[s], kb * BK, m0);
+            }
+          } else {
+            mbar_arrive_expect_tx(&wfull[s], L::WP_BYTES);
+            tma_load_2d(smem + L::OFF_WP + s * L::WP_BYTES, &tmW, &wfull[s], kb * (BK / 4), n0);
+          }
         }
       }
-      // Do not leave while copies into this CTA's shared memory are in flight.
-      const uint32_t inflight = it < S_TMA ? it : S_TMA;
+      // Do not leave while copies into this CTA's shared memory are in
+      // flight: the weight tiles signal wfull here; the even CTA also waits
+      // for the activation tiles of both CTAs (afull). The cluster barrier
+      // at exit keeps the odd CTA alive until then.
+      const uint32_t S = act ? S_TMA : S_W;
+      const uint32_t inflight = it < S ? it : S;
       for (uint32_t d = 0; d < inflight; ++d) {
         const uint32_t j = it - 1 - d;
-        mbar_wait(&full[j % S_TMA], (j / S_TMA) & 1, tmo, nullptr);
+        if (!act) mbar_wait(&wfull[j % S], (j / S) & 1, tmo, nullptr);
+        else if (leader) mbar_wait(&afull[j % S], (j / S) & 1, tmo, nullptr);
       }
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = FP4 ? make_idesc(1, 5, 5, BM, BN) : make_idesc(2, 1, 1, BM, BN);
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = FP4 ? make_idesc(1, 5, 5, TILE_M, BN) : make_idesc(2, 1, 1, TILE_M, BN);
       uint32_t it = 0, tl = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x, ++tl) {
+      for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride, ++tl) {
         const uint32_t acc = tl & 1, aph = (tl >> 1) & 1;
-        if (!mbar_wait(&tempty[acc], aph ^ 1, tmo, s_abort)) { fail(); break; }
+        if (!(PAIR ? mbar_wait_cluster(&tempty[acc], aph ^ 1, tmo, s_abort)
+                   : mbar_wait(&tempty[acc], aph ^ 1, tmo, s_abort))) { fail(); break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
           const uint32_t s = it % S_TMA, ph = (it / S_TMA) & 1;
           const uint32_t b = it % S_B, bph = (it / S_B) & 1;
-          if (!mbar_wait(&full[s], ph, tmo, s_abort) || !mbar_wait(&bfull[b], bph, tmo, s_abort)) {
-            fail(); ok = false; break;
-          }
+          const bool got = mbar_wait(&afull[s], ph, tmo, s_abort) &&
+                           (PAIR ? mbar_wait_cluster(&bfull[b], bph, tmo, s_abort)
+                                 : mbar_wait(&bfull[b], bph, tmo, s_abort));
+          if (!got) { fail(); ok = false; break; }
           tc_fence_after();
-          const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES);
-          const uint64_t bdesc = smem_desc_sw128(sB + b * B_BYTES);
 #pragma unroll
-          for (int k4 = 0; k4 < BK / 32; ++k4) {
-            // advance 32 bytes (2 x 16 B) along K inside the swizzled row
-            if (FP4) mma_f8f6f4(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, (kb | k4) != 0);
-            else     mma_i8(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, (kb | k4) != 0);
+          for (int kk = 0; kk < BK / 32; ++kk) {
+            // chunk kk / 4 of the k-block; advance 32 bytes (2 x 16 B) along K
+            // inside its swizzled 128-byte rows
+            const int sub = kk >> 2, k4 = kk & 3;
+            const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES + sub * SUB);
+            const uint64_t bdesc = smem_desc_sw128(sB + b * L::B_BYTES + sub * L::BROWS * 128);
+            const uint32_t accum = (kb | kk) != 0;
+            if (PAIR) {
+              if (FP4) mma_f8f6f4_pair(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, accum);
+              else     mma_i8_pair(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, accum);
+            } else {
+              if (FP4) mma_f8f6f4(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, accum);
+              else     mma_i8(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, accum);
+            }
           }
-          tc_commit(&empty[s]);
-          tc_commit(&bempty[b]);
+          if (PAIR) { tc_commit_pair_mc(&empty[s], 3); tc_commit_pair_mc(&bempty[b], 3); }
+          else      { tc_commit(&empty[s]); tc_commit(&bempty[b]); }
         }
-        if (ok) tc_commit(&tfull[acc]);
+        if (ok) {
+          if (PAIR) tc_commit_pair_mc(&tfull[acc], 3);
+          else      tc_commit(&tfull[acc]);
+        }
       }
-      tc_commit(mma_done);
+      if (PAIR) tc_commit_pair_mc(mma_done, 1);
+      else      tc_commit(mma_done);
       mbar_wait(mma_done, 0, tmo, nullptr);
     }
   } else if (warp >= 4 && warp < 8) {
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant
+    const uint32_t tempty_addr0 = lead(&tempty[0]);
+    const uint32_t stg = smem_u32(smem + L::OFF_STG) + q * 2048;  // this warp's staging block
+    float gam[8];  // every group's weight scale, loaded once
+#pragma unroll
+    for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
     uint32_t tl = 0;
-    for (int tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tl) {
-      const int m0 = (tile % p.tiles_m) * BM, n0 = (tile / p.tiles_m) * BN;
+    for (int tile = cta_slot; tile < p.num_tiles; tile += cta_stride, ++tl) {
+      const int m0 = (tile % p.tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+      const int n0 = (tile / p.tiles_m) * BN;
       const uint32_t acc = tl & 1, aph = (tl >> 1) & 1;
-      if (!mbar_wait(&tfull[acc], aph, tmo, s_abort)) { fail(); break; }
-      tc_fence_after();
       const int m = m0 + q * 32 + lane;
       const bool row_ok = m < p.M;
+      // the row scale is fetched before waiting, so its latency hides behind the mainloop
       const float xs_m = (row_ok && p.out_mode == kOutBf16) ? __ldg(p.xs + m) : 0.f;
+      if (!mbar_wait(&tfull[acc], aph, tmo, s_abort)) { fail(); break; }
+      tc_fence_after();
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int n = n0 + c * 32;
@@ -184,36 +258,69 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         uint32_t r[32];
         tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
         tmem_ld_wait();
-        if (!row_ok) continue;
         if (p.out_mode == kOutBf16) {
-          uint16_t* yrow = reinterpret_cast<uint16_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
-          float gm[32];
-          if (p.G == 1) {
-            const float g0 = __ldg(p.gamma);
+          // y = acc * (xs[m] * gamma[group(n)]); one scale per 32-column chunk
+          // unless the chunk straddles a group boundary
+          const int g0 = group_of(p, n);
+          const int g1 = group_of(p, min(n + 31, p.N - 1));
+          float s0 = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) gm[i] = g0;
+          for (int g = 0; g < 8; ++g) s0 = (g == g0) ? gam[g] : s0;
+          s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
+          float f[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
+            // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
+            // (1.5 * 2^23 + acc) - 1.5 * 2^23
+            f[i] = FP4 ? __uint_as_float(r[i])
+                       : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
+          }
+          if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] = __fmul_rn(f[i], s0);
           } else {
+            // the chunk crosses group boundaries: one pass per group touched
+            // (a dynamic loop, so the common path above is not predicated)
+#pragma unroll 1
+            for (int g = g0; g <= g1; ++g) {
+              const int lo = g == 0 ? 0 : p.group_end[g - 1], hi = p.group_end[g];
+              float t = 0.f;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) gm[i] = gamma_of(p, n + i);
-          }
+              for (int j = 0; j < 8; ++j) t = (j == g) ? gam[j] : t;
+              const float sg = __fmul_rn(xs_m, t);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            if (n + 8 * v >= p.N) break;
-            uint32_t w[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const int e = 8 * v + 2 * i;
-              float f0, f1;
-              if (FP4) { f0 = __uint_as_float(r[e]); f1 = __uint_as_float(r[e + 1]); }
-              else { f0 = static_cast<float>(static_cast<int32_t>(r[e]));
-                     f1 = static_cast<float>(static_cast<int32_t>(r[e + 1])); }
-              f0 = __fmul_rn(__fmul_rn(f0, xs_m), gm[e]);
-              f1 = __fmul_rn(__fmul_rn(f1, xs_m), gm[e + 1]);
-              w[i] = pack_bf16x2(f0, f1);
+              for (int i = 0; i < 32; ++i)
+                f[i] = (n + i >= lo && n + i < hi) ? __fmul_rn(f[i], sg) : f[i];
             }
-            reinterpret_cast<uint4*>(yrow)[v] = make_uint4(w[0], w[1], w[2], w[3]);
           }
-        } else {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
+          // stage the warp's 32 x 32 bf16 block (64 B per row, 16-byte units
+          // swizzled by row) and write it back as 64-byte row segments:
+          // store s covers rows 8s..8s+7, four lanes per row
+#pragma unroll
+          for (int v = 0; v < 4; ++v)
+            st_shared_v4(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4), w[4 * v], w[4 * v + 1],
+                         w[4 * v + 2], w[4 * v + 3]);
+          __syncwarp();
+          const int rr = lane >> 2, u = lane & 3;
+          uint4 o[4];
+#pragma unroll
+          for (int s2 = 0; s2 < 4; ++s2) {
+            const int row = 8 * s2 + rr;
+            o[s2] = ld_shared_v4(stg + row * 64 + ((u ^ ((row >> 1) & 3)) << 4));
+          }
+#pragma unroll
+          for (int s2 = 0; s2 < 4; ++s2) {
+            const int mm = m0 + q * 32 + 8 * s2 + rr;
+            if (mm < p.M && n + 8 * u < p.N)
+              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
+                                        static_cast<int64_t>(mm) * p.ldo + n + 8 * u) = o[s2];
+          }
+          __syncwarp();
+        } else if (row_ok) {
           uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
 #pragma unroll
           for (int v = 0; v < 8; ++v) {
@@ -224,46 +331,74 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
       tc_fence_before();
-      mbar_arrive(&tempty[acc]);
+      __syncwarp();
+      if (lane == 0) {  // one arrival per epilogue warp, on the even CTA
+        if (PAIR) mbar_arrive_cluster(tempty_addr0 + 8u * acc);
+        else      mbar_arrive(&tempty[acc]);
+      }
     }
   } else if (warp >= 8) {
     // ------------------------------------------------------------- unpack
     const int ut = threadIdx.x - 256;  // 0..255
+    const uint32_t bfull_addr0 = lead(&bfull[0]);
     uint32_t it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; ok && tile < p.num_tiles; tile += gridDim.x) {
+    for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride) {
       for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
-        const uint32_t s = it % S_TMA, ph = (it / S_TMA) & 1;
+        const uint32_t s = it % S_W, ph = (it / S_W) & 1;
         const uint32_t b = it % S_B, bph = (it / S_B) & 1;
-        if (!mbar_wait(&full[s], ph, tmo, s_abort) || !mbar_wait(&bempty[b], bph ^ 1, tmo, s_abort)) {
+        if (!mbar_wait(&wfull[s], ph, tmo, s_abort) || !mbar_wait(&bempty[b], bph ^ 1, tmo, s_abort)) {
           fail(); ok = false; break;
         }
-        const uint32_t src = sW + s * WP_BYTES;
-        const uint32_t dst = sB + b * B_BYTES;
+        const uint32_t src = sW + s * L::WP_BYTES;
+        const uint32_t dst = sB + b * L::B_BYTES;
+        constexpr int WPR = BK / 16;  // packed words per weight row
 #pragma unroll
-        for (int i = 0; i < (BN * BK / 16) / 256; ++i) {
-          const int w = ut + 256 * i;     // packed word index in the tile
-          const int n = w >> 3, j = w & 7;  // row, 16-byte chunk along K
+        for (int i = 0; i < (L::BROWS * WPR) / 256; ++i) {
+          const int w = ut + 256 * i;          // packed word index in the tile
+          const int n = w / WPR, j = w % WPR;  // row, 16-deep K group
+          const int sub = j >> 3, c = j & 7;   // 128-deep chunk, 16-byte column in it
           const uint32_t word = ld_shared_u32(src + 4 * w);
           const uint4 o = FP4 ? unpack16_e2m1(word) : unpack16_s8(word);
-          const uint32_t addr = dst + (n >> 3) * 1024 + (n & 7) * 128 + ((j ^ (n & 7)) << 4);
+          const uint32_t addr = dst + sub * (L::BROWS * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
+                                ((c ^ (n & 7)) << 4);
           st_shared_v4(addr, o.x, o.y, o.z, o.w);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&bfull[b]);
+        fence_proxy_async_smem();  // each thread's smem writes -> async proxy
+        __syncwarp();
+        if (lane == 0) {  // one arrival per unpack warp, on the even CTA
+          mbar_arrive(&wempty[s]);  // packed slot read: the weight producer may refill it
+          if (PAIR) mbar_arrive_cluster(bfull_addr0 + 8u * b);
+          else      mbar_arrive(&bfull[b]);
+        }
       }
     }
   }
 
   __syncthreads();
+  if (PAIR) cluster_sync();  // the pair's MMAs and remote arrivals are finished
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
-    tmem_dealloc(tmem_base, TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, TMEM_COLS);
+    else      tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
 }  // namespace gemm
+
+static cudaError_t make_map_3d(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
+                               const cuuint64_t (&dims)[3], const cuuint64_t (&strides)[2],
+                               const cuuint32_t (&box)[3], const char** why) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }
+  const cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(map, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) { *why = "cuTensorMapEncodeTiled rejected the activation layout"; return cudaErrorInvalidValue; }
+  return cudaSuccess;
+}
 
 static cudaError_t make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base,
                                uint64_t inner, uint64_t outer, uint64_t row_bytes,
@@ -282,18 +417,63 @@ static cudaError_t make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const v
   return cudaSuccess;
 }
 
+template <bool FP4, bool PAIR>
+static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const gemm::Params& p,
+                            cudaStream_t s) {
+  using namespace gemm;
+  auto kern = bitlinear_gemm_kernel<FP4, PAIR>;
+  static bool attr_set = false;  // once per process (not during graph capture)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         Layout<PAIR>::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int sms = num_sms();
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(THREADS);
+  cfg.dynamicSmemBytes = Layout<PAIR>::SMEM_BYTES;
+  cfg.stream = s;
+  if (PAIR) {
+    const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
+    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+  } else {
+    cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < sms ? p.num_tiles : sms));
+    cfg.numAttrs = 0;
+  }
+  return cudaLaunchKernelEx(&cfg, kern, tmA, tmW, p);
+}
+
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why) {
   using namespace gemm;
+  // CTA pairs once there are two 128-row halves to fill; their 3-D activation
+  // view needs whole 128-deep K chunks
+  const bool pair = a.M > BM && a.K % 128 == 0;
+  const int brows = pair ? BN / 2 : BN;
+  const int BK = pair ? Layout<true>::BK : Layout<false>::BK;
   CUtensorMap tmA, tmW;
   cudaError_t e;
-  if (fp4)
-    e = make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, a.xq, a.K, a.M, a.K / 2, BK, BM,
-                    CU_TENSOR_MAP_SWIZZLE_128B, why);
-  else
-    e = make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, a.K, a.M, a.K, BK, BM,
-                    CU_TENSOR_MAP_SWIZZLE_128B, why);
+  const CUtensorMapDataType adt = fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const uint64_t row_bytes = fp4 ? a.K / 2 : a.K;
+  if (pair) {
+    // [K/128 chunks][M rows][128 elements]: one box = 2 chunks x 128 rows,
+    // i.e. two standard 128-byte-swizzled 128 x 128 tiles back to back
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.M), static_cast<cuuint64_t>(a.K / 128)};
+    const cuuint64_t strides[2] = {row_bytes, fp4 ? 64u : 128u};
+    const cuuint32_t box[3] = {128, BM, static_cast<cuuint32_t>(Layout<true>::KSUB)};
+    e = make_map_3d(&tmA, adt, a.xq, dims, strides, box, why);
+  } else {
+    e = make_map_2d(&tmA, adt, a.xq, a.K, a.M, row_bytes, BK, BM, CU_TENSOR_MAP_SWIZZLE_128B, why);
+  }
   if (e != cudaSuccess) return e;
-  e = make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, a.K / 4, a.N, a.K / 4, BK / 4, BN,
+  e = make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, a.K / 4, a.N, a.K / 4, BK / 4, brows,
                   CU_TENSOR_MAP_SWIZZLE_NONE, why);
   if (e != cudaSuccess) return e;
 
@@ -302,7 +482,8 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
   p.num_kb = static_cast<int>((a.K + BK - 1) / BK);
-  p.tiles_m = static_cast<int>((a.M + BM - 1) / BM);
+  const int tile_m = pair ? 2 * BM : BM;
+  p.tiles_m = static_cast<int>((a.M + tile_m - 1) / tile_m);
   const int tiles_n = static_cast<int>((a.N + BN - 1) / BN);
   p.num_tiles = p.tiles_m * tiles_n;
   p.xs = a.xs;
@@ -315,16 +496,8 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
 
-  auto kern = fp4 ? bitlinear_gemm_kernel<true> : bitlinear_gemm_kernel<false>;
-  static bool attr_set[2] = {false, false};  // once per process (not during graph capture)
-  if (!attr_set[fp4 ? 1 : 0]) {
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set[fp4 ? 1 : 0] = true;
-  }
-  const int grid = p.num_tiles < num_sms() ? p.num_tiles : num_sms();
-  kern<<<grid, THREADS, SMEM_BYTES, s>>>(tmA, tmW, p);
-  return cudaGetLastError();
+  if (fp4) return pair ? launch_t<true, true>(tmA, tmW, p, s) : launch_t<true, false>(tmA, tmW, p, s);
+  return pair ? launch_t<false, true>(tmA, tmW, p, s) : launch_t<false, false>(tmA, tmW, p, s);
 }
 
 }  // namespace blt
