@@ -88,7 +88,7 @@ int bitlinear_ternarize_pack(const float* W, int64_t K, int64_t N, const int64_t
  *   x, up   device bf16 [M x ldx] (row stride ldx elements); up nullable
  *   q_out   device int8 [M x K] for INT8/INT4, uint8 [M x K/2] for FP4
  *   xs_out  device fp32 [M]
- * Requires K % 16 == 0, K <= 65536, ldx >= K, ldx % 8 == 0.
+ * Requires K % 16 == 0, K <= 49152, ldx >= K, ldx % 8 == 0.
  */
 int bitlinear_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, int64_t K, int64_t ldx,
                         int mode, void* q_out, float* xs_out, bitlinear_stream_t stream);
@@ -112,13 +112,14 @@ int bitlinear_topk_sparsify_i8(const uint16_t* x, int64_t M, int64_t K, int64_t 
  * BitLinear GEMM, ternary weights x 8-bit integer activation codes
  * ([A] abstract; [R] "Метод"), on tcgen05 tensor cores:
  *   acc[m,n] = sum_k xq[m,k] * W_t[k,n]                (exact int32)
- *   y[m,n]   = bf16_rne((float)acc * xs[m] * gamma[g(n)])  (two fp32 multiplies)
+ *   y[m,n]   = bf16_rne((float)acc * (xs[m] * gamma[g(n)]))  (fp32 multiplies)
  *   xq         device int8 [M x K], row stride K
  *   xs         device fp32 [M]
  *   Wp         device uint8 [N x K/4] from bitlinear_ternarize_pack
  *   gamma      device fp32 [G];  group_ends HOST int64 [G] (as for the pack)
  *   y          device bf16 [M x ldy]
- * Requires K % 64 == 0, N % 16 == 0, ldy >= N, ldy % 8 == 0, G in 1..8.
+ * Requires K % 64 == 0, K <= 32768 (|acc| < 2^22, converted exactly to fp32),
+ * N % 16 == 0, ldy >= N, ldy % 8 == 0, G in 1..8.
  * The w2a4 entry point takes INT4 codes ([-8, 7]) in int8 containers: sm_100
  * tensor cores have no 4-bit integer kind, so both run the s8 MMA.
  */
