@@ -137,9 +137,91 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
   (void)s_row;
 }
 
+// Rows of up to 4096 elements: one warp per row, the whole row held in
+// registers as bf16 (CPL 16-byte chunks per lane, all loads in flight at
+// once), warp-shuffle absmax, no shared memory and no block barrier.
+template <int MODE, bool RELU2, int CPL>
+__global__ void __launch_bounds__(kQuantThreads) quant_act_warp_kernel(
+    const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int64_t M, int K,
+    int64_t ldx, void* __restrict__ q_out, float* __restrict__ xs_out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t m = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
+  if (m >= M) return;  // whole warp
+  const int nchunk = K >> 3;
+  const uint4* xr = reinterpret_cast<const uint4*>(x + m * ldx);
+  const uint4* ur = reinterpret_cast<const uint4*>(RELU2 ? up + m * ldx : x);
+  uint4 xv[CPL], uv[RELU2 ? CPL : 1];
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    const int c = lane + 32 * j;
+    xv[j] = c < nchunk ? __ldg(xr + c) : make_uint4(0, 0, 0, 0);
+    if (RELU2) uv[j] = c < nchunk ? __ldg(ur + c) : make_uint4(0, 0, 0, 0);
+  }
+  auto row_vals = [&](int j, float (&h)[8]) {
+    bf16x8_to_f32(xv[j], h);
+    if (RELU2) {
+      float u[8];
+      bf16x8_to_f32(uv[RELU2 ? j : 0], u);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float r = h[i] > 0.f ? h[i] : 0.f;
+        h[i] = __fmul_rn(__fmul_rn(r, r), u[i]);
+      }
+    }
+  };
+  float amax = 0.f;
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    float h[8];
+    row_vals(j, h);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(h[i]));
+  }
+  amax = warp_max(amax);
+  constexpr float Q = MODE == BITLINEAR_MODE_INT8 ? 127.f : (MODE == BITLINEAR_MODE_INT4 ? 7.f : 6.f);
+  const float a = fmaxf(amax, kEps);
+  const float inv = __fdiv_rn(Q, a);
+  if (lane == 0) xs_out[m] = __fdiv_rn(a, Q);
+#pragma unroll
+  for (int j = 0; j < CPL; ++j) {
+    const int c = lane + 32 * j;
+    if (c >= nchunk) break;
+    float h[8];
+    row_vals(j, h);
+    if (MODE == BITLINEAR_MODE_FP4) {
+      float v[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(h[i], inv);
+      reinterpret_cast<uint32_t*>(q_out)[m * nchunk + c] = cvt_e2m1x8(v);
+    } else {
+      int q[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) q[i] = quant_code(h[i], inv, -Q - 1.f, Q);
+      reinterpret_cast<uint2*>(q_out)[m * nchunk + c] =
+          make_uint2(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]));
+    }
+  }
+}
+
+template <int MODE, bool RELU2, int CPL>
+static cudaError_t launch_quant_warp(const uint16_t* x, const uint16_t* up, int64_t M, int K,
+                                     int64_t ldx, void* q, float* xs, cudaStream_t s) {
+  constexpr int RPB = kQuantThreads / 32;
+  quant_act_warp_kernel<MODE, RELU2, CPL><<<static_cast<unsigned>((M + RPB - 1) / RPB),
+                                            kQuantThreads, 0, s>>>(x, up, M, K, ldx, q, xs);
+  return cudaGetLastError();
+}
+
 template <int MODE, bool RELU2>
 static cudaError_t launch_quant_t(const uint16_t* x, const uint16_t* up, int64_t M, int K,
                                   int64_t ldx, void* q, float* xs, cudaStream_t s) {
+  const int chunks_per_lane = (K / 8 + 31) / 32;
+  if (chunks_per_lane <= 1) return launch_quant_warp<MODE, RELU2, 1>(x, up, M, K, ldx, q, xs, s);
+  if (chunks_per_lane <= 2) return launch_quant_warp<MODE, RELU2, 2>(x, up, M, K, ldx, q, xs, s);
+  if (chunks_per_lane <= 4) return launch_quant_warp<MODE, RELU2, 4>(x, up, M, K, ldx, q, xs, s);
+  if (chunks_per_lane <= 8) return launch_quant_warp<MODE, RELU2, 8>(x, up, M, K, ldx, q, xs, s);
+  if (!RELU2 && chunks_per_lane <= 16)
+    return launch_quant_warp<MODE, RELU2, 16>(x, up, M, K, ldx, q, xs, s);
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
   auto kern = quant_act_kernel<MODE, RELU2>;
   static int attr_bytes = 48 * 1024;  // raised once, monotonically (outside graph capture in practice)
@@ -308,78 +390,100 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 // G = D/8 threads of one (token, head) row reduce their absmax with a
 // segmented warp shuffle. A warp covers 32/G whole rows whose 3-bit
 // streams (3 bytes per thread) form 96 contiguous bytes, staged in shared
-// memory and written as 24 aligned words.
+// memory and written as 24 aligned words. The list of 4-bit tokens is copied
+// to shared memory once per block (up to kKeepSmem entries) and searched
+// there; row -> (token, head) uses 32-bit division.
+constexpr int kKeepSmem = 1024;
+constexpr int KV_TILES = 4;  // warp tiles per warp (16-byte loads in flight per thread)
+
 template <int G>
 __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
-    const uint16_t* __restrict__ kv, int64_t rows, int64_t H, const int32_t* __restrict__ keep4,
+    const uint16_t* __restrict__ kv, uint32_t rows, uint32_t H, const int32_t* __restrict__ keep4,
     int n4, uint8_t* __restrict__ codes3, uint8_t* __restrict__ codes4, float* __restrict__ scale) {
   constexpr int D = 8 * G;
+  constexpr int RPW = 32 / G;  // rows per warp tile
   __shared__ __align__(16) uint8_t stage[kQuantThreads / 32][96];
+  __shared__ int32_t s_keep[kKeepSmem];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
-  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * kQuantThreads + threadIdx.x;
-  const int64_t row = gtid / G;
-  const int g = static_cast<int>(gtid % G);
-  const bool valid = row < rows;
-
-  float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-  if (valid) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kv + row * D) + g), f);
-  float amax = 0.f;
+  const int n4s = n4 < kKeepSmem ? n4 : kKeepSmem;
+  for (int i = threadIdx.x; i < n4s; i += kQuantThreads) s_keep[i] = __ldg(keep4 + i);
+  const int g = lane % G;
+  // this warp's KV_TILES consecutive warp tiles: all loads issued up front
+  const uint32_t tile0 = (blockIdx.x * (kQuantThreads / 32) + wid) * KV_TILES;
+  float f[KV_TILES][8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+  for (int j = 0; j < KV_TILES; ++j) {
+    const uint32_t row = (tile0 + j) * RPW + lane / G;
 #pragma unroll
-  for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-
-  const int64_t t = row / H, h = row % H;
-  int j = -1;  // index of t among the 4-bit tokens
-  if (valid) {
-    int lo = 0, hi = n4 - 1;
-    while (lo <= hi) {
-      const int mid = (lo + hi) >> 1;
-      const int p = __ldg(keep4 + mid);
-      if (p == t) { j = mid; break; }
-      if (p < t) lo = mid + 1; else hi = mid - 1;
+    for (int i = 0; i < 8; ++i) f[j][i] = 0.f;
+    if (row < rows) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kv + static_cast<size_t>(row) * D) + g), f[j]);
+  }
+  __syncthreads();  // s_keep ready
+#pragma unroll
+  for (int j = 0; j < KV_TILES; ++j) {
+    const uint32_t warp_row0 = (tile0 + j) * RPW;
+    const uint32_t row = warp_row0 + lane / G;
+    const bool valid = row < rows;
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[j][i]));
+#pragma unroll
+    for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const uint32_t t = row / H, h = row - t * H;
+    int jk = -1;  // index of t among the 4-bit tokens
+    if (valid && n4 > 0) {
+      int lo = 0, hi = n4 - 1;
+      while (lo <= hi) {
+        const int mid = (lo + hi) >> 1;
+        const int p = mid < kKeepSmem ? s_keep[mid] : __ldg(keep4 + mid);
+        if (p == static_cast<int>(t)) { jk = mid; break; }
+        if (p < static_cast<int>(t)) lo = mid + 1; else hi = mid - 1;
+      }
     }
-  }
-  const bool four = j >= 0;
-  const float Q = four ? 7.f : 3.f;
-  const float a = fmaxf(amax, kEps);
-  const float inv = __fdiv_rn(Q, a);
-  const float lo_c = four ? -8.f : -4.f, hi_c = four ? 7.f : 3.f;
-  uint32_t packed3 = 0u, packed4 = 0u;
+    const bool four = jk >= 0;
+    const float Q = four ? 7.f : 3.f;
+    const float a = fmaxf(amax, kEps);
+    const float inv = __fdiv_rn(Q, a);
+    uint32_t packed3 = 0u;
+    if (four) {
+      uint32_t packed4 = 0u;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int c = quant_code(f[i], inv, lo_c, hi_c);
-    packed3 |= static_cast<uint32_t>(c + 4) << (3 * i);
-    packed4 |= static_cast<uint32_t>(c + 8) << (4 * i);
+      for (int i = 0; i < 8; ++i)
+        packed4 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -8.f, 7.f) + 8) << (4 * i);
+      if (valid)
+        reinterpret_cast<uint32_t*>(codes4 + (static_cast<size_t>(jk) * H + h) * (D / 2))[g] = packed4;
+    } else {
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        packed3 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -4.f, 3.f) + 4) << (3 * i);
+    }
+    if (valid && g == 0) scale[row] = __fdiv_rn(a, Q);
+    stage[wid][3 * lane + 0] = static_cast<uint8_t>(packed3);
+    stage[wid][3 * lane + 1] = static_cast<uint8_t>(packed3 >> 8);
+    stage[wid][3 * lane + 2] = static_cast<uint8_t>(packed3 >> 16);
+    __syncwarp();
+    const int64_t rows_here = static_cast<int64_t>(rows) - warp_row0;
+    const int nbytes = rows_here >= RPW ? 96 : static_cast<int>(rows_here > 0 ? rows_here : 0) * 3 * G;
+    if (lane * 4 < nbytes)
+      reinterpret_cast<uint32_t*>(codes3 + static_cast<size_t>(warp_row0) * (3 * G))[lane] =
+          reinterpret_cast<const uint32_t*>(stage[wid])[lane];
+    __syncwarp();
   }
-  if (four) packed3 = 0u;
-  if (valid && four)
-    reinterpret_cast<uint32_t*>(codes4 + (static_cast<int64_t>(j) * H + h) * (D / 2))[g] = packed4;
-  if (valid && g == 0) scale[row] = __fdiv_rn(a, Q);
-
-  stage[wid][3 * lane + 0] = static_cast<uint8_t>(packed3);
-  stage[wid][3 * lane + 1] = static_cast<uint8_t>(packed3 >> 8);
-  stage[wid][3 * lane + 2] = static_cast<uint8_t>(packed3 >> 16);
-  __syncwarp();
-  const int64_t warp_row0 = (gtid - lane) / G;
-  const int64_t rows_here = rows - warp_row0;
-  const int nbytes = rows_here >= 32 / G ? 96 : static_cast<int>(rows_here > 0 ? rows_here : 0) * 3 * G;
-  if (lane * 4 < nbytes)
-    reinterpret_cast<uint32_t*>(codes3 + warp_row0 * (3 * G))[lane] =
-        reinterpret_cast<const uint32_t*>(stage[wid])[lane];
 }
 
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s) {
-  const int64_t rows = T * H;
+  const uint32_t rows = static_cast<uint32_t>(T * H);  // the entry point bounds rows * G < 2^32
   const int G = static_cast<int>(D / 8);
-  const int64_t threads = rows * G;
-  const unsigned grid = static_cast<unsigned>((threads + kQuantThreads - 1) / kQuantThreads);
+  const uint64_t threads = static_cast<uint64_t>(rows) * G;
+  const uint64_t per_block = static_cast<uint64_t>(kQuantThreads) * KV_TILES;
+  const unsigned grid = static_cast<unsigned>((threads + per_block - 1) / per_block);
   const int n = static_cast<int>(n4);
-  if (G == 8) kv_quant_kernel<8><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
-  else if (G == 16) kv_quant_kernel<16><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
-  else kv_quant_kernel<32><<<grid, kQuantThreads, 0, s>>>(kv, rows, H, keep4, n, codes3, codes4, scale);
+  const uint32_t h = static_cast<uint32_t>(H);
+  if (G == 8) kv_quant_kernel<8><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
+  else if (G == 16) kv_quant_kernel<16><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
+  else kv_quant_kernel<32><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
   return cudaGetLastError();
 }
 
