@@ -69,6 +69,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--seed", type=int, default=1)
+    ap.add_argument("--no-overlap", action="store_true",
+                    help="launch without programmatic dependent launch (each kernel waits for "
+                         "the previous one before it starts)")
     ap.add_argument("--section", default=None,
                     help="run only one breakdown section (o_proj, down_proj, decode, kv), e.g. "
                          "to profile its kernels; prints that section's JSON")
@@ -208,17 +211,27 @@ class PrefillReplica:
                   for k, n in (("qkv4", 3 * D), ("gu4", 2 * FFN), ("qkvf", 3 * D), ("guf", 2 * FFN))}
 
 
+def gemm_call(B, r: PrefillReplica, name):
+    """Launch one of the step's four GEMMs on replica r."""
+    if name == "w2a4_qkv":
+        B.gemm_w2a4(r.q4, r.xs4, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkv4"])
+    elif name == "w2a4_gu":
+        B.gemm_w2a4(r.q4, r.xs4, r.gu[0], r.gu[1], GU[1], y=r.y["gu4"])
+    elif name == "w2fp4_qkv":
+        B.gemm_w2fp4(r.f4, r.xsf, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkvf"])
+    else:
+        B.gemm_w2fp4(r.f4, r.xsf, r.gu[0], r.gu[1], GU[1], y=r.y["guf"])
+
+
 def run_step(B, r: PrefillReplica, ev=None):
-    """One step; ev (optional) = dict of (start, end) event pairs per GEMM."""
-    def rec(name, i):
-        if ev is not None:
-            ev[name][i].record()
+    """One step: INT4 quantiser, its two GEMMs, FP4 quantiser, its two GEMMs
+    (ev is unused: steps are timed whole)."""
     B.quant_act(r.x, B.MODE_INT4, out=r.q4, xs=r.xs4)
-    rec("w2a4_qkv", 0); B.gemm_w2a4(r.q4, r.xs4, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkv4"]); rec("w2a4_qkv", 1)
-    rec("w2a4_gu", 0); B.gemm_w2a4(r.q4, r.xs4, r.gu[0], r.gu[1], GU[1], y=r.y["gu4"]); rec("w2a4_gu", 1)
+    gemm_call(B, r, "w2a4_qkv")
+    gemm_call(B, r, "w2a4_gu")
     B.quant_act(r.x, B.MODE_FP4, out=r.f4, xs=r.xsf)
-    rec("w2fp4_qkv", 0); B.gemm_w2fp4(r.f4, r.xsf, r.qkv[0], r.qkv[1], QKV[1], y=r.y["qkvf"]); rec("w2fp4_qkv", 1)
-    rec("w2fp4_gu", 0); B.gemm_w2fp4(r.f4, r.xsf, r.gu[0], r.gu[1], GU[1], y=r.y["guf"]); rec("w2fp4_gu", 1)
+    gemm_call(B, r, "w2fp4_qkv")
+    gemm_call(B, r, "w2fp4_gu")
 
 
 LAUNCHES_PER_STEP = 6
@@ -236,9 +249,11 @@ def make_prefill(B, torch, dev, seed, with_oracle_inputs=False):
     return d, qkv, gu
 
 
-def graph_set(torch, stream, steps_fns, names, E):
+def graph_set(torch, stream, steps_fns, names, E, timed=True):
     """Capture E copies of each replica's step as CUDA graphs, each copy with
-    its own external timing events around the named launches."""
+    its own external timing events around the named launches (timed=False:
+    no event nodes, for whole-step timing; event nodes inside a graph
+    serialise the work around them and add their own cost)."""
     graphs, events = [], []
     with torch.cuda.stream(stream):
         for fn in steps_fns:  # run once eagerly (first-call set-up outside capture)
@@ -247,7 +262,7 @@ def graph_set(torch, stream, steps_fns, names, E):
     for _ in range(E):
         for fn in steps_fns:
             ev = {n: (torch.cuda.Event(enable_timing=True, external=True),
-                      torch.cuda.Event(enable_timing=True, external=True)) for n in names}
+                      torch.cuda.Event(enable_timing=True, external=True)) for n in names} if timed else None
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=stream):
                 fn(ev)
@@ -282,10 +297,22 @@ def run_graphs(torch, stream, graphs, events, names, steps, warmup, ws=1, clocks
     ms = max_over_ranks(t0.elapsed_time(t1), ws)
     last = min(steps, NG)
     kms = {}
-    for n in names:
+    for n in (names if events[0] is not None else ()):
         v = [events[j][n][0].elapsed_time(events[j][n][1]) for j in range(NG - last, NG)]
         kms[n] = statistics.mean(v)
     return ms, kms, clk
+
+
+def time_calls(torch, stream, calls, steps, warm, per_graph=8):
+    """Mean device time (ms) of one call: graphs of `per_graph` back-to-back
+    calls cycling over `calls` (one closure per buffer replica), no event
+    nodes inside, timed as a whole over `steps` graph replays."""
+    n = len(calls)
+    fns = [(lambda ev, i=i: [calls[(i + j) % n]() for j in range(per_graph)]) for i in range(n)]
+    gs, es = graph_set(torch, stream, fns, (), max(1, 8 // n), timed=False)
+    ms, _, _ = run_graphs(torch, stream, gs, es, (), steps, warm)
+    del gs
+    return ms / steps / per_graph
 
 
 def bench_ours(args, ws, rank, local):
@@ -294,17 +321,24 @@ def bench_ours(args, ws, rank, local):
     dev = f"cuda:{local}"
     torch.cuda.set_device(local)
     B.lib()
+    B.set_launch_overlap(not args.no_overlap)
     d, qkv, gu = make_prefill(B, torch, dev, args.seed)
     R = 3
     reps = [PrefillReplica(B, torch, d["x"], qkv, gu, dev) for _ in range(R)]
     stream = torch.cuda.Stream(device=dev)
     fns = [(lambda ev, r=r: run_step(B, r, ev)) for r in reps]
-    graphs, events = graph_set(torch, stream, fns, GEMM_NAMES, E=8)
+    # whole-step timing: graphs without event nodes
+    graphs, events = graph_set(torch, stream, fns, GEMM_NAMES, E=8, timed=False)
     B.check_status(stream=stream)
-    ms, kms, clk = run_graphs(torch, stream, graphs, events, GEMM_NAMES, args.steps, args.warmup,
-                              ws, ClockSampler(local))
+    ms, _, clk = run_graphs(torch, stream, graphs, events, GEMM_NAMES, args.steps, args.warmup,
+                            ws, ClockSampler(local))
     B.check_status(stream=stream)
     del graphs
+    # per-kernel durations: each GEMM alone, back to back over the replicas
+    ksteps, kwarm = min(args.steps, 240), max(3, args.warmup // 4)
+    kms = {n: time_calls(torch, stream, [(lambda r=r, n=n: gemm_call(B, r, n)) for r in reps],
+                         ksteps, kwarm) for n in GEMM_NAMES}
+    B.check_status(stream=stream)
 
     peaks, peak_src = load_peaks()
     int8_peak = RATIO_INT8 * peaks["bf16_tflops"]
@@ -315,7 +349,9 @@ def bench_ours(args, ws, rank, local):
                 "achieved": round(ach, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
                 "frac": round(ach / int8_peak, 4), "traffic": traffic, "traffic_source": tsrc,
                 "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TF/s x {RATIO_INT8} "
-                               "(nominal int8/bf16 dense ratio)"}
+                               "(nominal int8/bf16 dense ratio)",
+                "timing": "the GEMM alone: CUDA graphs of 8 back-to-back launches over the 3 replicas, "
+                          "CUDA events on the launching stream"}
     kernels = {}
     for n in GEMM_NAMES:
         tops = GEMM_OPS[n] / (kms[n] * 1e-3) / 1e12
@@ -333,7 +369,8 @@ def bench_ours(args, ws, rank, local):
                       "gate_up_out": 2 * FFN, "variants": ["INT4 (s8 MMA)", "FP4 e2m1 (f8f6f4 MMA)"],
                       "parallelism": f"replicas x{ws}",
                       "l2": f"{R} rotating replicas of all inputs/weights/outputs (>270 MB > 126 MB L2)",
-                      "graphs": "one CUDA graph per step"},
+                      "graphs": "one CUDA graph per step",
+                      "launch_overlap": not args.no_overlap},
            "roofline": roofline, "kernels": kernels, "clocks": clk,
            "gpu_launches": LAUNCHES_PER_STEP * args.steps}
     return out, (d, qkv, gu, reps, B, torch, dev, stream)
@@ -485,7 +522,8 @@ SECTIONS = ("o_proj", "down_proj", "decode", "kv")
 
 def breakdown(ctx, args, sections=SECTIONS):
     """The other workloads of the path, each timed the same way (rotating
-    replicas larger than L2, CUDA graphs, per-launch events)."""
+    replicas larger than L2, CUDA graphs without event nodes; a kernel's time
+    is that of a graph of back-to-back launches of it alone)."""
     B, torch, dev, stream = ctx[4], ctx[5], ctx[6], ctx[7]
     peaks, src = load_peaks()
     out = {"peaks": f"{src}: HBM {peaks['hbm_gbs']} GB/s, int8 {RATIO_INT8 * peaks['bf16_tflops']:.0f} "
@@ -512,14 +550,17 @@ def section_o_proj(B, torch, dev, stream, peaks, steps, warm):
                          xs=torch.empty(M, dtype=torch.float32, device=dev),
                          y=torch.empty((M, N), dtype=torch.bfloat16, device=dev)))
 
+    def topk(b): B.topk_sparsify_i8(b["x"], out=b["q"], xs=b["xs"])
+    def gemm(b): B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
+
     def o_step(ev, b):
-        if ev: ev["topk"][0].record()
-        B.topk_sparsify_i8(b["x"], out=b["q"], xs=b["xs"])
-        if ev: ev["topk"][1].record(); ev["gemm"][0].record()
-        B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
-        if ev: ev["gemm"][1].record()
-    gs, es = graph_set(torch, stream, [(lambda ev, b=b: o_step(ev, b)) for b in bufs], ("topk", "gemm"), 8)
-    ms, k, _ = run_graphs(torch, stream, gs, es, ("topk", "gemm"), steps, warm)
+        topk(b)
+        gemm(b)
+    gs, es = graph_set(torch, stream, [(lambda ev, b=b: o_step(ev, b)) for b in bufs], (), 8, timed=False)
+    ms, _, _ = run_graphs(torch, stream, gs, es, (), steps, warm)
+    del gs
+    k = {"topk": time_calls(torch, stream, [(lambda b=b: topk(b)) for b in bufs], steps, warm),
+         "gemm": time_calls(torch, stream, [(lambda b=b: gemm(b)) for b in bufs], steps, warm)}
     ops = 2 * M * K * N
     tb = M * K * 2 + M * K + M * 4
     out["o_proj_topk_w2a8_4096x4096x4096"] = {
@@ -546,14 +587,22 @@ def section_down_proj(B, torch, dev, stream, peaks, steps, warm):
              y=torch.empty((M, N), dtype=torch.bfloat16, device=dev))
     del dn
 
+    b2 = dict(b, q=torch.empty_like(b["q"]), y=torch.empty_like(b["y"]), Wp=b["Wp"].clone())
+
+    def quant(b): B.quant_act(b["gate"], B.MODE_INT8, up=b["up"], out=b["q"], xs=b["xs"])
+    def gemm(b): B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
+
     def d_step(ev):
-        if ev: ev["quant"][0].record()
-        B.quant_act(b["gate"], B.MODE_INT8, up=b["up"], out=b["q"], xs=b["xs"])
-        if ev: ev["quant"][1].record(); ev["gemm"][0].record()
-        B.gemm_w2a8(b["q"], b["xs"], b["Wp"], b["g"], (N,), y=b["y"])
-        if ev: ev["gemm"][1].record()
-    gs, es = graph_set(torch, stream, [d_step], ("quant", "gemm"), 24)
-    ms, k, _ = run_graphs(torch, stream, gs, es, ("quant", "gemm"), steps, warm)
+        quant(b)
+        gemm(b)
+    gs, es = graph_set(torch, stream, [d_step], (), 24, timed=False)
+    ms, _, _ = run_graphs(torch, stream, gs, es, (), steps, warm)
+    del gs
+    quant(b2)
+    # gate/up (180 MB) exceed L2 on their own; the GEMM alone alternates two
+    # sets of codes/weights/outputs (2 x 88 MB)
+    k = {"quant": time_calls(torch, stream, [lambda: quant(b)], steps, warm),
+         "gemm": time_calls(torch, stream, [lambda: gemm(b), lambda: gemm(b2)], steps, warm)}
     ops = 2 * M * K * N
     qb = 2 * M * K * 2 + M * K + M * 4
     zero_codes = float((b["q"] == 0).float().mean().item())
@@ -568,7 +617,7 @@ def section_down_proj(B, torch, dev, stream, peaks, steps, warm):
 
 
 def section_decode(B, torch, dev, stream, peaks, steps, warm):
-    """Decode: one LLaMA-7B-shaped layer at batch 1 / 8 / 64 (weight GB/s).
+    """Decode: one LLaMA-7B-shaped layer at batch 1 / 4 / 8 / 64 (weight GB/s).
 
     The projections that share an input run as one launch with per-group
     scales (q|k|v: N = 12288, 3 groups; gate|up: N = 22016, 2 groups), then
@@ -594,7 +643,7 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
             for _ in range(R)]
     names = tuple(shapes)
     dec = {}
-    for batch in (1, 8, 64):
+    for batch in (1, 4, 8, 64):
         x = _dev_bf16(torch, lay["x"][:batch], dev)
         xo = _dev_bf16(torch, lay["xo"][:batch], dev)
         ga = _dev_bf16(torch, lay["gate"][:batch], dev)
@@ -607,33 +656,37 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
         qd = torch.empty((batch, F), dtype=torch.int8, device=dev)
         xsd = torch.empty(batch, dtype=torch.float32, device=dev)
 
-        def gemv(ev, name, xq, xs, wr):
-            if ev: ev[name][0].record()
-            B.gemv_w2(xq, xs, wr[name][0], wr[name][1], shapes[name][2], y=ys[name])
-            if ev: ev[name][1].record()
+        ins = {"qkv": (q4, xs4), "o": (qo, xso), "gate_up": (q4, xs4), "down": (qd, xsd)}
+
+        def gemv(name, r):
+            xq, xs = ins[name]
+            B.gemv_w2(xq, xs, wdev[r][name][0], wdev[r][name][1], shapes[name][2], y=ys[name])
 
         def l_step(ev, r):
-            wr = wdev[r]
             B.quant_act(x, B.MODE_INT4, out=q4, xs=xs4)
-            gemv(ev, "qkv", q4, xs4, wr)
+            gemv("qkv", r)
             B.topk_sparsify_i8(xo, out=qo, xs=xso)
-            gemv(ev, "o", qo, xso, wr)
-            gemv(ev, "gate_up", q4, xs4, wr)
+            gemv("o", r)
+            gemv("gate_up", r)
             B.quant_act(ga, B.MODE_INT8, up=up, out=qd, xs=xsd)
-            gemv(ev, "down", qd, xsd, wr)
-        gs, es = graph_set(torch, stream, [(lambda ev, r=r: l_step(ev, r)) for r in range(R)], names, 4)
-        ms, k, _ = run_graphs(torch, stream, gs, es, names, steps, warm)
+            gemv("down", r)
+        gs, es = graph_set(torch, stream, [(lambda ev, r=r: l_step(ev, r)) for r in range(R)], (), 4,
+                           timed=False)
+        ms, _, _ = run_graphs(torch, stream, gs, es, (), steps, warm)
+        del gs
+        k = {n: time_calls(torch, stream, [(lambda n=n, r=r: gemv(n, r)) for r in range(R)], steps, warm)
+             for n in names}
         gemv_ms = sum(k.values())
         per = {n: {"us": round(k[n] * 1e3, 2), "GBps": round(K_ * N_ // 4 / k[n] / 1e6, 1)}
                for n, (K_, N_, _) in shapes.items()}
         dec[f"batch{batch}"] = {
             "layer_step_us": round(ms / steps * 1e3, 2),
             "gemv_sum_us": round(gemv_ms * 1e3, 2),
+            "gemv_sum_note": "each projection timed alone, back to back over 6 weight replicas",
             "weight_GBps": round(wbytes / gemv_ms / 1e6, 1),
             "weight_frac_hbm": round(wbytes / gemv_ms / 1e6 / hbm, 4),
             "layer_weight_GBps_incl_quantisers": round(wbytes / (ms / steps) / 1e6, 1),
             "per_projection": per}
-        del gs, es
     out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=7,
                                        gemv_launches="qkv (fused, 3 groups), o, gate_up (fused, 2 groups), down",
                                        **dec)
@@ -653,13 +706,10 @@ def section_kv(B, torch, dev, stream, peaks, steps, warm):
     o4 = [torch.empty((1, H, Dh // 2), dtype=torch.uint8, device=dev) for _ in range(2)]
     sc = [torch.empty((T, H), dtype=torch.float32, device=dev) for _ in range(2)]
 
-    def kv_step(ev, r):
-        if ev: ev["kv"][0].record()
+    def kv_step(r):
         for j in range(2):
             B.kv_quant_3bit(kvs[r][j], keep, codes3=o3[j], codes4=o4[j], scale=sc[j])
-        if ev: ev["kv"][1].record()
-    gs, es = graph_set(torch, stream, [(lambda ev, r=r: kv_step(ev, r)) for r in range(4)], ("kv",), 6)
-    ms, k, _ = run_graphs(torch, stream, gs, es, ("kv",), steps, warm)
+    k = {"kv": time_calls(torch, stream, [(lambda r=r: kv_step(r)) for r in range(4)], steps, warm)}
     kb = 2 * (T * H * Dh * 2 + T * H * 3 * Dh // 8 + T * H * 4 + H * Dh // 2)
     out["kv_quant_3bit_2x4096x32x128"] = {"us": round(k["kv"] * 1e3, 2),
                                          "GBps": round(kb / k["kv"] / 1e6, 1),
@@ -675,6 +725,7 @@ def main():
         import bit_quantised_gemm_b200 as B
         torch.cuda.set_device(local)
         B.lib()
+        B.set_launch_overlap(not args.no_overlap)
         stream = torch.cuda.Stream(device=f"cuda:{local}")
         ctx = (None, None, None, None, B, torch, f"cuda:{local}", stream)
         print(json.dumps(breakdown(ctx, args, (args.section,))), flush=True)

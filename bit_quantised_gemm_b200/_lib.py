@@ -38,6 +38,7 @@ _SIGS = {
     "bitlinear_last_error": ([], _c.c_char_p),
     "bitlinear_version": ([], _INT),
     "bitlinear_set_wait_timeout_ns": ([_I64], _INT),
+    "bitlinear_set_launch_overlap": ([_INT], _INT),
     "bitlinear_ternarize_pack": ([_P, _I64, _I64, _P, _INT, _P, _P], _INT),
     "bitlinear_quant_act": ([_P, _P, _I64, _I64, _I64, _INT, _P, _P, _P], _INT),
     "bitlinear_topk_sparsify_i8": ([_P, _I64, _I64, _I64, _I64, _P, _P, _P, _P], _INT),
@@ -124,6 +125,11 @@ def status_buffer(device=None) -> torch.Tensor:
 # ------------------------------------------------------------------ API
 def version() -> int:
     return lib().bitlinear_version()
+
+
+def set_launch_overlap(enable: bool):
+    """Programmatic dependent launch for later calls (see bitlinear.h)."""
+    _check(lib().bitlinear_set_launch_overlap(1 if enable else 0))
 
 
 def set_wait_timeout_ns(ns: int):

@@ -1,5 +1,6 @@
 // C ABI entry points: argument validation on the host, then one launch on
 // the caller's stream. The library allocates no device memory.
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -15,6 +16,7 @@ namespace {
 
 thread_local char g_err[512] = "";
 int64_t g_timeout_ns = 2000000000LL;
+std::atomic<bool> g_overlap{false};
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -116,6 +118,8 @@ int num_sms() {
   return n;
 }
 
+bool launch_overlap() { return g_overlap.load(std::memory_order_relaxed); }
+
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s) {
   wait_probe_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
   return cudaGetLastError();
@@ -127,7 +131,12 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 100; }
+int bitlinear_version(void) { return 101; }
+
+int bitlinear_set_launch_overlap(int enable) {
+  g_overlap.store(enable != 0);
+  return ok();
+}
 
 int bitlinear_set_wait_timeout_ns(int64_t ns) {
   if (ns <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "timeout must be positive");
@@ -282,6 +291,10 @@ int bitlinear_gemv_w2(const int8_t* xq, const float* xs, const uint8_t* Wp, cons
   a.ldo = ldy;
   a.out_mode = blt::kOutBf16;
   a.status = dev_status;
+  if (blt::gemv_dp4a_supported(M, K)) {
+    cudaError_t e = blt::launch_gemv_dp4a(a, stream);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2 (dp4a)");
+  }
   const char* why = nullptr;
   cudaError_t e = blt::launch_gemv(a, stream, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2", why);
@@ -298,8 +311,8 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
   if (!kv || !codes3 || !scale) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: null pointer");
   if (!aligned16(kv) || !aligned16(codes3) || (codes4 && !aligned16(codes4)))
     return fail(BITLINEAR_ERR_ALIGNMENT, "kv_quant_3bit: pointers must be 16-byte aligned");
-  if (T * H > (1LL << 40)) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: too large");
-  if (T == 0) return ok();
+  if (T * H * (D / 8) >= (1LL << 32) - 256 || n_keep4 > 0x7FFFFFFF)
+    return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: T * H * D / 8 must stay below 2^32");
   cudaError_t e = blt::launch_kv_quant(kv, T, H, D, keep4_pos, n_keep4, codes3, codes4, scale, stream);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_quant_3bit launch");
 }

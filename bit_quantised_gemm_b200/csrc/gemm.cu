@@ -129,6 +129,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (PAIR) cluster_sync();  // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  // Only now (TMEM held) may the next kernel in the stream start its CTAs.
+  pdl_trigger();
 
   const uint32_t sA = smem_u32(smem + L::OFF_A);
   const uint32_t sB = smem_u32(smem + L::OFF_B);
@@ -148,6 +150,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // ----------------------------------------- TMA producers (A: warp 0, W: warp 2)
     if (lane == 0) {
       const bool act = warp == 0;
+      // activation codes come from the previous kernel; packed weights do not
+      if (act) pdl_wait();
       uint32_t it = 0;
       bool ok = true;
       for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride) {
@@ -240,6 +244,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     float gam[8];  // every group's weight scale, loaded once
 #pragma unroll
     for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
+    pdl_wait();  // row scales come from the previous kernel; y may still be read by it
     uint32_t tl = 0;
     for (int tile = cta_slot; tile < p.num_tiles; tile += cta_stride, ++tl) {
       const int m0 = (tile % p.tiles_m) * TILE_M + static_cast<int>(rank) * BM;
@@ -430,25 +435,13 @@ static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, cons
     attr_set = true;
   }
   const int sms = num_sms();
-  cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = Layout<PAIR>::SMEM_BYTES;
-  cfg.stream = s;
   if (PAIR) {
     const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
-    cfg.gridDim = dim3(static_cast<unsigned>(2 * pairs));
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-  } else {
-    cfg.gridDim = dim3(static_cast<unsigned>(p.num_tiles < sms ? p.num_tiles : sms));
-    cfg.numAttrs = 0;
+    return launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS),
+                         Layout<PAIR>::SMEM_BYTES, s, 2u, tmA, tmW, p);
   }
-  return cudaLaunchKernelEx(&cfg, kern, tmA, tmW, p);
+  return launch_kernel(kern, dim3(static_cast<unsigned>(p.num_tiles < sms ? p.num_tiles : sms)),
+                       dim3(THREADS), Layout<PAIR>::SMEM_BYTES, s, 0u, tmA, tmW, p);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why) {

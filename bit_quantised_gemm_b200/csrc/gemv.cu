@@ -116,6 +116,7 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  pdl_trigger();  // TMEM is held: the next kernel in the stream may start
   const uint64_t tmo = p.timeout_ns;
   const uint32_t sA = smem_u32(smem + OFF_A);
   const uint32_t sX = smem_u32(smem + OFF_X);
@@ -130,6 +131,9 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
     // -------------------------------------------- TMA (weights: warp 0, activations: warp 2)
     if (lane == 0) {
       const bool wts = warp == 0;
+      // activation codes come from the previous kernel (the row scales and y
+      // are touched after the block-wide barrier that follows this wait)
+      if (!wts) pdl_wait();
       int issued = 0;
       for (int j = 0; j < nsup; ++j, ++issued) {
         const uint32_t s = j % S, ph = (j / S) & 1;
@@ -310,19 +314,8 @@ cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(tiles * c));
-  cfg.blockDim = dim3(THREADS);
-  cfg.dynamicSmemBytes = SMEM_BYTES;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = static_cast<unsigned>(c);
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, bitlinear_gemv_kernel, tmX, tmW, p);
+  return launch_kernel(bitlinear_gemv_kernel, dim3(static_cast<unsigned>(tiles * c)), dim3(THREADS),
+                       SMEM_BYTES, s, static_cast<unsigned>(c), tmX, tmW, p);
 }
 
 }  // namespace blt

@@ -1,0 +1,407 @@
+// Decode-time BitLinear for a few tokens (up to 8) on the CUDA cores.
+//
+// With up to eight tokens the layer is a matrix-vector product whose cost is
+// streaming the 2-bit weights out of HBM (N x K/4 bytes): every weight meets
+// at most eight activation codes, and the tensor cores would only add an
+// unpack round trip through shared memory. This kernel keeps the weight
+// stream in flight with bulk copies and does the arithmetic with 4-way byte
+// dot products (dp4a) on the packed codes themselves, without expanding them
+// to int8 first.
+//
+// Arithmetic. The packed word j of a weight row holds codes c = W_t + 1 in
+// {0, 1, 2}; element 16j + 8h + i sits at bits [4i+2h, 4i+2h+2). With
+// t = w >> 2, the four masks
+//     w & 0x03030303 -> c of elements 16j + {0, 2, 4, 6}        (x1)
+//     t & 0x03030303 -> c of elements 16j + {8, 10, 12, 14}     (x1)
+//     w & 0x30303030 -> c of elements 16j + {1, 3, 5, 7}        (x16)
+//     t & 0x30303030 -> c of elements 16j + {9, 11, 13, 15}     (x16)
+// leave one code per byte, so dp4a against the activation bytes regrouped in
+// that order gives sum_k c[k] x[k] in two integer accumulators (scales 1 and
+// 16). The layer output is acc = sum_k x[k] W_t[k] = sum_k c[k] x[k] - sum_k
+// x[k], exact in int32, followed by the usual epilogue
+//     y = bf16_rne((float)acc * (xs[m] * gamma[g(n)])).
+//
+// Work split. Rows of Wp are contiguous (K/4 bytes each), so an item of RW
+// consecutive output features is one contiguous range, fetched with a single
+// cp.async.bulk into a per-warp ring of SW slots. Items are dealt round-robin
+// over all warps of the grid (neighbouring warps read neighbouring rows). A
+// lane takes the packed words j = lane, lane + 32, ... of every row of the
+// item, so the 4-byte weight reads of a warp and its 16-byte reads of the
+// activation codes (all MT tokens, held in shared memory for the whole
+// kernel) are contiguous. The RW x MT partial sums of a lane are reduced
+// across the warp with a transposing butterfly: log2(RW MT) exchange steps
+// that halve the values held per lane, then plain xor steps.
+#include <algorithm>
+
+#include "common.cuh"
+#include "launch.h"
+#include "ptx.cuh"
+
+namespace blt {
+namespace gemv_cc {
+
+constexpr int SW = 2;         // ring slots per warp
+constexpr int MAX_WARPS = 16;
+constexpr int SMEM_LIMIT = 232448;
+
+struct Params {
+  int M, N, K;
+  int n_items;
+  const int8_t* xq;
+  const float* xs;
+  const uint8_t* Wp;
+  const float* gamma;
+  int G;
+  int group_end[8];
+  uint16_t* y;
+  int64_t ldy;
+  int* status;
+  uint64_t timeout_ns;
+};
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+      ::"r"(dst), "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// Regroup 16 activation bytes x0..x15 (little-endian words a, b, c, d) into
+// {x0,x2,x4,x6}, {x8,x10,x12,x14}, {x1,x3,x5,x7}, {x9,x11,x13,x15}: the
+// element order of the four code masks above.
+__device__ __forceinline__ uint4 regroup16(uint4 v) {
+  uint4 r;
+  r.x = __byte_perm(v.x, v.y, 0x6420);
+  r.y = __byte_perm(v.z, v.w, 0x6420);
+  r.z = __byte_perm(v.x, v.y, 0x7531);
+  r.w = __byte_perm(v.z, v.w, 0x7531);
+  return r;
+}
+
+// Sum of the four signed bytes of each word.
+__device__ __forceinline__ int byte_sum16(uint4 v) {
+  int s = __dp4a(static_cast<int>(v.x), 0x01010101, 0);
+  s = __dp4a(static_cast<int>(v.y), 0x01010101, s);
+  s = __dp4a(static_cast<int>(v.z), 0x01010101, s);
+  return __dp4a(static_cast<int>(v.w), 0x01010101, s);
+}
+
+// Butterfly over the 32 lanes: on return v[0] holds the warp-wide sum of
+// value number `idx`, and every lane of a group of 32 / NV consecutive lanes
+// holds the same one (idx runs over 0..NV-1 with the group).
+template <int NV>
+__device__ __forceinline__ int transpose_reduce(int (&v)[NV], int lane, int& idx) {
+  static_assert(NV >= 1 && NV <= 32 && (NV & (NV - 1)) == 0, "power of two up to 32");
+  idx = 0;
+#pragma unroll
+  for (int step = 0; (NV >> (step + 1)) >= 1; ++step) {
+    const int h = NV >> (step + 1);
+    const int o = 16 >> step;
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int j = 0; j < h; ++j) {
+      const int send = up ? v[j] : v[j + h];
+      const int keep = up ? v[j + h] : v[j];
+      v[j] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, o);
+    }
+    if (up) idx += h;
+  }
+  int s = v[0];
+#pragma unroll
+  for (int o = 16 / NV; o >= 1; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  return s;
+}
+
+// dp4a with unsigned bytes in a (the masked codes reach 128) and signed
+// bytes in b (the activation codes).
+__device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
+  int d;
+  asm("dp4a.u32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+  return d;
+}
+
+// One packed word against the MT tokens' regrouped activation words.
+// NACC = 4: four masks without a shift, accumulators at scales 1, 4, 16, 64
+// (fewest instructions; used for one or two tokens). NACC = 2: one shift,
+// accumulators at scales 1 and 16 (half the registers).
+template <int MT, int NACC>
+__device__ __forceinline__ void word_dot(uint32_t w, const uint4 (&xv)[MT], int (&acc)[MT][NACC]) {
+  if constexpr (NACC == 4) {
+    const uint32_t m0 = w & 0x03030303u, m1 = w & 0x0C0C0C0Cu;
+    const uint32_t m2 = w & 0x30303030u, m3 = w & 0xC0C0C0C0u;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      acc[t][0] = dp4a_us(m0, xv[t].x, acc[t][0]);
+      acc[t][1] = dp4a_us(m1, xv[t].y, acc[t][1]);
+      acc[t][2] = dp4a_us(m2, xv[t].z, acc[t][2]);
+      acc[t][3] = dp4a_us(m3, xv[t].w, acc[t][3]);
+    }
+  } else {
+    const uint32_t sh = w >> 2;
+    const uint32_t m0 = w & 0x03030303u, m1 = sh & 0x03030303u;
+    const uint32_t m2 = w & 0x30303030u, m3 = sh & 0x30303030u;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      acc[t][0] = dp4a_us(m0, xv[t].x, acc[t][0]);
+      acc[t][0] = dp4a_us(m1, xv[t].y, acc[t][0]);
+      acc[t][1] = dp4a_us(m2, xv[t].z, acc[t][1]);
+      acc[t][1] = dp4a_us(m3, xv[t].w, acc[t][1]);
+    }
+  }
+}
+
+// sum_k c[k] x[k] from the scaled accumulators (each is a multiple of its
+// scale, so the shifts are exact).
+template <int NACC>
+__device__ __forceinline__ int combine(const int (&a)[NACC]) {
+  if constexpr (NACC == 4) return a[0] + (a[1] >> 2) + (a[2] >> 4) + (a[3] >> 6);
+  else return a[0] + (a[1] >> 4);
+}
+
+template <int MT, int RW>
+__global__ void __launch_bounds__(MAX_WARPS * 32, 1)
+bitlinear_gemv_dp4a_kernel(const Params p) {
+  constexpr int NACC = MT <= 2 ? 4 : 2;
+  constexpr int U = MT <= 2 ? 4 : (MT == 4 ? 2 : 1);  // words per lane per batch of loads
+  constexpr int NV = RW * MT;
+  extern __shared__ __align__(16) uint8_t smem[];
+  const int K = p.K;
+  const int row_bytes = K >> 2;
+  const int slot_bytes = RW * row_bytes;
+  const int nwarps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  uint8_t* xsm = smem;                                  // [MT][K] regrouped codes
+  uint8_t* ring = smem + MT * K;                        // [nwarps][SW][slot_bytes]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(ring + nwarps * SW * slot_bytes);
+  uint64_t* xbar = bars + nwarps * SW;
+  int* xsum = reinterpret_cast<int*>(xbar + 1);         // [MT]
+
+  uint8_t* my_ring = ring + warp * SW * slot_bytes;
+  uint64_t* my_bar = bars + warp * SW;
+  const int gw = blockIdx.x * nwarps + warp;
+  const int GW = gridDim.x * nwarps;
+  const int n_mine = gw < p.n_items ? (p.n_items - 1 - gw) / GW + 1 : 0;
+
+  auto issue = [&](int s) {  // lane 0: fetch the s-th item of this warp
+    const int item = gw + s * GW;
+    const int n0 = item * RW;
+    const int rows = min(RW, p.N - n0);
+    const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
+    uint64_t* bar = my_bar + (s % SW);
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load(smem_u32(my_ring + (s % SW) * slot_bytes),
+              p.Wp + static_cast<int64_t>(n0) * row_bytes, bytes, bar);
+  };
+
+  // The weight stream does not depend on the previous kernel in the stream:
+  // the first items of every warp go out before waiting for it.
+  if (lane == 0) {
+    for (int i = 0; i < SW; ++i) mbar_init(my_bar + i, 1);
+    if (threadIdx.x == 0) mbar_init(xbar, 1);
+    fence_mbar_init();
+    for (int s = 0; s < min(SW, n_mine); ++s) issue(s);
+  }
+  float gam[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) gam[i] = i < p.G ? __ldg(p.gamma + i) : 0.f;
+  pdl_trigger();
+  pdl_wait();  // activation codes and scales come from the previous kernel
+  if (threadIdx.x == 0) {  // the codes are one contiguous M x K block
+    const uint32_t xbytes = static_cast<uint32_t>(p.M * K);
+    mbar_arrive_expect_tx(xbar, xbytes);
+    bulk_load(smem_u32(xsm), p.xq, xbytes, xbar);
+  }
+  float xsc[MT];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) xsc[t] = t < p.M ? __ldg(p.xs + t) : 0.f;
+  if (threadIdx.x < MT) xsum[threadIdx.x] = 0;
+  // tokens p.M .. MT-1 are zero codes
+  for (int i = p.M * K / 16 + threadIdx.x; i < MT * K / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(xsm)[i] = make_uint4(0u, 0u, 0u, 0u);
+  __syncthreads();
+
+  // Regroup the codes in place and take their row sums.
+  const bool x_ok = mbar_wait(xbar, 0, p.timeout_ns, nullptr);
+  if (x_ok) {
+    const int groups = p.M * K / 16;
+    int part[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) part[t] = 0;
+    for (int i = threadIdx.x; i < groups; i += blockDim.x) {
+      uint4* q = reinterpret_cast<uint4*>(xsm) + i;
+      const uint4 v = *q;
+      const int t = i / (K / 16);
+      const int bs = byte_sum16(v);
+#pragma unroll
+      for (int u = 0; u < MT; ++u) part[u] += (u == t) ? bs : 0;
+      *q = regroup16(v);
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) part[t] += __shfl_xor_sync(0xFFFFFFFFu, part[t], o);
+      if (lane == 0 && part[t] != 0) atomicAdd(&xsum[t], part[t]);
+    }
+  }
+  __syncthreads();
+  int xsm_sum[MT];
+#pragma unroll
+  for (int t = 0; t < MT; ++t) xsm_sum[t] = xsum[t];
+
+  const uint32_t x_base = smem_u32(xsm);
+  const int words = K >> 4;
+  bool timed_out = !x_ok;
+  int s = 0;
+  for (; s < n_mine && !timed_out; ++s) {
+    if (!mbar_wait(my_bar + (s % SW), (s / SW) & 1, p.timeout_ns, nullptr)) {
+      timed_out = true;
+      break;
+    }
+    const uint32_t w_base = smem_u32(my_ring + (s % SW) * slot_bytes);
+    int acc[RW][MT][NACC];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int t = 0; t < MT; ++t)
+#pragma unroll
+        for (int a = 0; a < NACC; ++a) acc[r][t][a] = 0;
+
+    // U words per lane are loaded before any arithmetic; words past the row
+    // end read as code 0, which adds nothing.
+    for (int j0 = lane; j0 < words; j0 += 32 * U) {
+      uint4 xv[U][MT];
+      uint32_t w[U][RW];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + 32 * u;
+        const bool in = j < words;
+#pragma unroll
+        for (int t = 0; t < MT; ++t)
+          xv[u][t] = in ? ld_shared_v4(x_base + t * K + 16 * j) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (int r = 0; r < RW; ++r) w[u][r] = in ? ld_shared_u32(w_base + r * row_bytes + 4 * j) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int r = 0; r < RW; ++r) word_dot<MT, NACC>(w[u][r], xv[u], acc[r]);
+    }
+    __syncwarp();  // every lane has read the slot
+    if (lane == 0 && s + SW < n_mine) issue(s + SW);
+
+    int v[NV];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+      for (int t = 0; t < MT; ++t) v[r * MT + t] = combine<NACC>(acc[r][t]);
+    int idx;
+    const int sum = transpose_reduce<NV>(v, lane, idx);
+    if ((lane & (32 / NV - 1)) == 0) {
+      const int r = idx / MT, t = idx % MT;
+      const int n = (gw + s * GW) * RW + r;
+      if (t < p.M && n < p.N) {
+        int ts = 0;
+        float xst = 0.f;
+#pragma unroll
+        for (int u = 0; u < MT; ++u) {
+          ts = (u == t) ? xsm_sum[u] : ts;
+          xst = (u == t) ? xsc[u] : xst;
+        }
+        int g = 0;
+#pragma unroll
+        for (int i = 0; i < 7; ++i) g += (i < p.G - 1 && n >= p.group_end[i]) ? 1 : 0;
+        float gm = gam[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) gm = (g == i) ? gam[i] : gm;
+        const int acc = sum - ts;
+        p.y[static_cast<int64_t>(t) * p.ldy + n] = __bfloat16_as_ushort(
+            __float2bfloat16_rn(static_cast<float>(acc) * (xst * gm)));
+      }
+    }
+  }
+  if (timed_out) {
+    report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
+    // Let copies still in flight land before the block's shared memory is
+    // released (bounded as well).
+    if (lane == 0)
+      for (int q = s; q < min(s + SW, n_mine); ++q)
+        mbar_wait(my_bar + (q % SW), (q / SW) & 1, p.timeout_ns, nullptr);
+    if (threadIdx.x == 0 && !x_ok) mbar_wait(xbar, 0, p.timeout_ns, nullptr);
+    __syncwarp();
+  }
+}
+
+}  // namespace gemv_cc
+
+static size_t dp4a_smem_bytes(int mt, int rw, int64_t K, int warps) {
+  return size_t(mt) * K + size_t(warps) * gemv_cc::SW * rw * (K / 4) +
+         size_t(warps) * gemv_cc::SW * 8 + 8 + 8 * 4;
+}
+
+static int dp4a_tokens(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 4 ? 4 : 8; }
+
+// Largest warp count (<= 16) whose ring fits next to the activation codes;
+// 0 when even one warp does not fit.
+static int dp4a_warps_fit(int mt, int rw, int64_t K) {
+  for (int w = gemv_cc::MAX_WARPS; w >= 1; --w)
+    if (dp4a_smem_bytes(mt, rw, K, w) <= size_t(gemv_cc::SMEM_LIMIT)) return w;
+  return 0;
+}
+
+bool gemv_dp4a_supported(int64_t M, int64_t K) {
+  if (M < 1 || M > kGemvDp4aMaxTokens || K % 64 != 0) return false;
+  return dp4a_warps_fit(dp4a_tokens(M), 2, K) > 0;
+}
+
+template <int MT, int RW>
+static cudaError_t launch_mt(gemv_cc::Params p, cudaStream_t s) {
+  p.n_items = (p.N + RW - 1) / RW;
+  const int grid = std::min(num_sms(), p.n_items);
+  int warps = (p.n_items + grid - 1) / grid;
+  warps = std::min(warps, dp4a_warps_fit(MT, RW, p.K));
+  const size_t smem = dp4a_smem_bytes(MT, RW, p.K, warps);
+  auto kern = gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  return launch_kernel(kern, dim3(grid), dim3(warps * 32), smem, s, 0u, p);
+}
+
+// Items of 4 output features when there are enough of them to give every
+// SM a full complement of warps (and the ring fits), else of 2.
+template <int MT>
+static cudaError_t launch_pick_rows(const gemv_cc::Params& p, cudaStream_t s) {
+  if constexpr (MT <= 4) {  // eight tokens: 2 rows (registers)
+    if (int64_t(p.N) >= int64_t(4) * gemv_cc::MAX_WARPS * num_sms() &&
+        dp4a_warps_fit(MT, 4, p.K) == gemv_cc::MAX_WARPS)
+      return launch_mt<MT, 4>(p, s);
+  }
+  return launch_mt<MT, 2>(p, s);
+}
+
+cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s) {
+  gemv_cc::Params p{};
+  p.M = static_cast<int>(a.M);
+  p.N = static_cast<int>(a.N);
+  p.K = static_cast<int>(a.K);
+  p.xq = static_cast<const int8_t*>(a.xq);
+  p.xs = a.xs;
+  p.Wp = a.Wp;
+  p.gamma = a.gamma;
+  p.G = a.G;
+  for (int i = 0; i < 8; ++i) p.group_end[i] = a.group_end[i];
+  p.y = static_cast<uint16_t*>(a.out);
+  p.ldy = a.ldo;
+  p.status = a.status;
+  p.timeout_ns = a.timeout_ns;
+  switch (dp4a_tokens(a.M)) {
+    case 1: return launch_pick_rows<1>(p, s);
+    case 2: return launch_pick_rows<2>(p, s);
+    case 4: return launch_pick_rows<4>(p, s);
+    default: return launch_pick_rows<8>(p, s);
+  }
+}
+
+}  // namespace blt

@@ -39,6 +39,11 @@ struct GemmArgs {
 // encoder is unavailable (message in *why).
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why);
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why);
+// CUDA-core decode path for few tokens (dp4a on packed codes); larger
+// batches take the tensor-core GEMV.
+constexpr int kGemvDp4aMaxTokens = 8;
+bool gemv_dp4a_supported(int64_t M, int64_t K);
+cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s);
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once at run time.
@@ -48,5 +53,40 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn get_encode_tiled();
 int num_sms();
+
+// Process-wide switch (bitlinear_set_launch_overlap): launch with
+// programmatic stream serialisation so a kernel may start while the previous
+// one in the stream finishes. Every kernel calls pdl_wait() before it reads
+// activations or scales or writes an output.
+bool launch_overlap();
+
+// Launch with the overlap attribute (when on) and, for cluster_x > 0, a
+// cluster of cluster_x CTAs along x.
+template <typename... Exp, typename... Act>
+inline cudaError_t launch_kernel(void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem,
+                                 cudaStream_t s, unsigned cluster_x, Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[2];
+  unsigned n = 0;
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  if (cluster_x > 0) {
+    attr[n].id = cudaLaunchAttributeClusterDimension;
+    attr[n].val.clusterDim.x = cluster_x;
+    attr[n].val.clusterDim.y = 1;
+    attr[n].val.clusterDim.z = 1;
+    ++n;
+  }
+  if (launch_overlap()) {
+    attr[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+  }
+  cfg.attrs = attr;
+  cfg.numAttrs = n;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Act&&>(args)...);
+}
 
 }  // namespace blt

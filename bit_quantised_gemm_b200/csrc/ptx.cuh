@@ -31,6 +31,12 @@ __device__ __forceinline__ uint32_t elect_one() {
 }
 
 // ------------------------------------------------------------- mbarriers
+// Programmatic dependent launch: wait for the grids this one depends on to
+// complete (a no-op when the launch did not allow overlap), and let the next
+// grid in the stream start its own prologue.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)
                : "memory");

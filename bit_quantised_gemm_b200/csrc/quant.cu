@@ -6,6 +6,7 @@
 // an IEEE fp32 operation (explicit __fdiv_rn / __fmul_rn, rintf = RNE).
 #include "common.cuh"
 #include "launch.h"
+#include "ptx.cuh"
 
 namespace blt {
 
@@ -85,6 +86,8 @@ template <int MODE, bool RELU2>
 __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int K, int64_t ldx,
     void* __restrict__ q_out, float* __restrict__ xs_out) {
+  pdl_wait();  // inputs come from the previous kernel in the stream
+  pdl_trigger();
   extern __shared__ float4 s_row4[];
   float* s_row = reinterpret_cast<float*>(s_row4);
   __shared__ float red[kQuantThreads / 32];
@@ -144,6 +147,8 @@ template <int MODE, bool RELU2, int CPL>
 __global__ void __launch_bounds__(kQuantThreads) quant_act_warp_kernel(
     const uint16_t* __restrict__ x, const uint16_t* __restrict__ up, int64_t M, int K,
     int64_t ldx, void* __restrict__ q_out, float* __restrict__ xs_out) {
+  pdl_wait();  // inputs come from the previous kernel in the stream
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int64_t m = static_cast<int64_t>(blockIdx.x) * (kQuantThreads / 32) + (threadIdx.x >> 5);
   if (m >= M) return;  // whole warp
@@ -207,9 +212,9 @@ template <int MODE, bool RELU2, int CPL>
 static cudaError_t launch_quant_warp(const uint16_t* x, const uint16_t* up, int64_t M, int K,
                                      int64_t ldx, void* q, float* xs, cudaStream_t s) {
   constexpr int RPB = kQuantThreads / 32;
-  quant_act_warp_kernel<MODE, RELU2, CPL><<<static_cast<unsigned>((M + RPB - 1) / RPB),
-                                            kQuantThreads, 0, s>>>(x, up, M, K, ldx, q, xs);
-  return cudaGetLastError();
+  return launch_kernel(quant_act_warp_kernel<MODE, RELU2, CPL>,
+                       dim3(static_cast<unsigned>((M + RPB - 1) / RPB)), dim3(kQuantThreads), 0, s, 0u,
+                       x, up, M, K, ldx, q, xs);
 }
 
 template <int MODE, bool RELU2>
@@ -231,8 +236,8 @@ static cudaError_t launch_quant_t(const uint16_t* x, const uint16_t* up, int64_t
     if (e != cudaSuccess) return e;
     attr_bytes = static_cast<int>(smem);
   }
-  kern<<<static_cast<unsigned>(M), kQuantThreads, smem, s>>>(x, up, K, ldx, q, xs);
-  return cudaGetLastError();
+  return launch_kernel(kern, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), smem, s, 0u,
+                       x, up, K, ldx, q, xs);
 }
 
 cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, int64_t K,
@@ -259,6 +264,8 @@ template <int E>
 __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
     const uint16_t* __restrict__ x, int K, int64_t ldx, int k, int8_t* __restrict__ q_out,
     float* __restrict__ xs_out, uint8_t* __restrict__ mask_out) {
+  pdl_wait();  // inputs come from the previous kernel in the stream
+  pdl_trigger();
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sums[8];
   __shared__ float red[8];
@@ -374,15 +381,13 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                            int8_t* q, float* xs, uint8_t* mask, cudaStream_t s) {
   const int kk = static_cast<int>(k), KK = static_cast<int>(K);
   const unsigned grid = static_cast<unsigned>(M);
-  if (K <= 8 * kQuantThreads)
-    topk_i8_kernel<8><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
-  else if (K <= 16 * kQuantThreads)
-    topk_i8_kernel<16><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
-  else if (K <= 32 * kQuantThreads)
-    topk_i8_kernel<32><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
-  else
-    topk_i8_kernel<64><<<grid, kQuantThreads, 0, s>>>(x, KK, ldx, kk, q, xs, mask);
-  return cudaGetLastError();
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, dim3(grid), dim3(kQuantThreads), 0, s, 0u, x, KK, ldx, kk, q, xs, mask);
+  };
+  if (K <= 8 * kQuantThreads) return go(topk_i8_kernel<8>);
+  if (K <= 16 * kQuantThreads) return go(topk_i8_kernel<16>);
+  if (K <= 32 * kQuantThreads) return go(topk_i8_kernel<32>);
+  return go(topk_i8_kernel<64>);
 }
 
 // ------------------------------------------------------------ KV 3-bit
@@ -400,6 +405,8 @@ template <int G>
 __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
     const uint16_t* __restrict__ kv, uint32_t rows, uint32_t H, const int32_t* __restrict__ keep4,
     int n4, uint8_t* __restrict__ codes3, uint8_t* __restrict__ codes4, float* __restrict__ scale) {
+  pdl_wait();  // inputs come from the previous kernel in the stream
+  pdl_trigger();
   constexpr int D = 8 * G;
   constexpr int RPW = 32 / G;  // rows per warp tile
   __shared__ __align__(16) uint8_t stage[kQuantThreads / 32][96];
@@ -481,10 +488,13 @@ cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
   const unsigned grid = static_cast<unsigned>((threads + per_block - 1) / per_block);
   const int n = static_cast<int>(n4);
   const uint32_t h = static_cast<uint32_t>(H);
-  if (G == 8) kv_quant_kernel<8><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
-  else if (G == 16) kv_quant_kernel<16><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
-  else kv_quant_kernel<32><<<grid, kQuantThreads, 0, s>>>(kv, rows, h, keep4, n, codes3, codes4, scale);
-  return cudaGetLastError();
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, dim3(grid), dim3(kQuantThreads), 0, s, 0u, kv, rows, h, keep4, n,
+                         codes3, codes4, scale);
+  };
+  if (G == 8) return go(kv_quant_kernel<8>);
+  if (G == 16) return go(kv_quant_kernel<16>);
+  return go(kv_quant_kernel<32>);
 }
 
 }  // namespace blt

@@ -184,6 +184,18 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
  * BITLINEAR_ERR_TIMEOUT if a kernel gave up a bounded wait. */
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream);
 
+/*
+ * Launch overlap (programmatic dependent launch), process-wide, default off.
+ * When enabled, later launches may start while the previous kernel in the
+ * same stream is still running: each kernel first does the work that needs
+ * only the weights (Wp, gamma: loads into shared memory, barrier and tensor
+ * memory set-up) and waits for that previous kernel to complete before it
+ * reads activation codes, inputs or scales, or writes any output. Enable it
+ * only when no call's Wp or gamma is written by the kernel just before it in
+ * its stream. A CUDA graph keeps the setting in force when it was captured.
+ */
+int bitlinear_set_launch_overlap(int enable);
+
 /* Limit (ns) on every in-kernel wait of later launches; default 2e9. */
 int bitlinear_set_wait_timeout_ns(int64_t ns);
 

@@ -185,7 +185,8 @@ def test_bitlinear_layer_end_to_end(mode, M, N, K, groups):
     assert_bf16_close(bits(y), y_o)
 
 
-@pytest.mark.parametrize("M", [1, 8, 17, 64])
+# M <= 8 runs the CUDA-core (dp4a) path, larger M the tensor-core path.
+@pytest.mark.parametrize("M", [1, 2, 3, 4, 6, 8, 9, 17, 64])
 @pytest.mark.parametrize("N,K", [(128, 128), (4096, 4096), (4096, 11008), (1024, 512)])
 def test_gemv_parity(M, N, K):
     rng = np.random.default_rng(M + N + K)
@@ -198,9 +199,41 @@ def test_gemv_parity(M, N, K):
     assert_bf16_close(bits(y), y_o)
 
 
-def test_gemv_matches_gemm():
+@pytest.mark.parametrize("M,N,K", [(1, 12288, 4096), (4, 22016, 4096)])
+def test_gemv_decode_full_size(M, N, K):
+    """Fused q/k/v and gate/up projections of the decode layer at full size."""
+    rng = np.random.default_rng(N + M)
+    xq = rng.integers(-8, 8, size=(M, K)).astype(np.int8)
+    xs = rng.uniform(0.01, 1, M).astype(np.float32)
+    groups = (N // 3, 2 * N // 3, N) if N % 3 == 0 else (N // 2, N)
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, groups, 13)
+    y = B.gemv_w2(torch.from_numpy(xq).to(DEV), torch.from_numpy(xs).to(DEV), Wp, gamma_d, groups)
+    B.check_status()
+    _, y_o = O.bitlinear_int(xq, xs, Wt, gamma, groups)
+    assert_bf16_close(bits(y), y_o)
+
+
+def test_gemv_extreme_codes():
+    """All codes at -128 against all-+1 / all--1 weight rows: the largest
+    accumulators the decode path can see at K = 11008."""
+    M, N, K = 2, 256, 11008
+    xq = np.full((M, K), -128, dtype=np.int8)
+    xs = np.ones(M, dtype=np.float32)
+    Wf = np.where((np.arange(N) % 2) == 0, 1.0, -1.0)[None, :].repeat(K, 0).astype(np.float32)
+    Wf[:, 5] = 0.0
+    Wt, gamma = O.ternarize(Wf, (N,))
+    Wp = torch.from_numpy(O.pack_ternary(Wt)).to(DEV)
+    y = B.gemv_w2(torch.from_numpy(xq).to(DEV), torch.from_numpy(xs).to(DEV), Wp,
+                  torch.from_numpy(gamma).to(DEV), (N,))
+    B.check_status()
+    _, y_o = O.bitlinear_int(xq, xs, Wt, gamma, (N,))
+    assert_bf16_close(bits(y), y_o)
+
+
+@pytest.mark.parametrize("M", [1, 3, 33])
+def test_gemv_matches_gemm(M):
     rng = np.random.default_rng(3)
-    M, N, K = 33, 2048, 2048
+    N, K = 2048, 2048
     xq = torch.from_numpy(rng.integers(-8, 8, size=(M, K)).astype(np.int8)).to(DEV)
     xs = torch.from_numpy(rng.uniform(0.01, 1, M).astype(np.float32)).to(DEV)
     _, _, Wp, gamma_d = prep_weights(K, N, (1024, 2048), 12)
@@ -244,3 +277,50 @@ def test_library_prep_feeds_gpu_gemm():
     xq_o, xs_o = O.quant_act(d["x"], O.MODE_INT4)
     _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, (256,))
     assert_bf16_close(bits(y), y_o)
+
+
+def _dependent_chain(x_dec, x_pre, wts):
+    """Kernels that each read the output of the one just before them:
+    decode (quantiser -> GEMV -> quantiser -> GEMV -> top-k -> GEMV) and
+    prefill (quantiser -> GEMM -> top-k -> GEMM -> KV quantiser)."""
+    (Wp1, g1), (Wp2, g2), (Wp3, g3) = wts
+    outs = []
+    q, xs = B.quant_act(x_dec, O.MODE_INT4)
+    y = B.gemv_w2(q, xs, Wp1, g1, (1024,))
+    q, xs = B.quant_act(y, O.MODE_INT8)
+    y = B.gemv_w2(q, xs, Wp2, g2, (1024,))
+    q, xs = B.topk_sparsify_i8(y)[:2]
+    outs.append(B.gemv_w2(q, xs, Wp3, g3, (1024,)))
+    q, xs = B.quant_act(x_pre, O.MODE_INT4)
+    y = B.gemm_w2a4(q, xs, Wp1, g1, (1024,))
+    q, xs = B.topk_sparsify_i8(y)[:2]
+    y = B.gemm_w2a8(q, xs, Wp2, g2, (1024,))
+    outs.append(y)
+    codes3, _, scale = B.kv_quant_3bit(y.view(-1, 8, 128), None)
+    outs += [codes3, scale]
+    return [o.clone() for o in outs]
+
+
+@pytest.mark.parametrize("M", [1, 6, 40])
+def test_launch_overlap_dependent_chain(M):
+    """With launch overlap on, every kernel must still see its producer's
+    finished output: the chain gives the same bits as with overlap off."""
+    wts = [prep_weights(1024, 1024, (1024,), 30 + i)[2:] for i in range(3)]
+    runs = []
+    for overlap in (False, True, True):
+        B.set_launch_overlap(overlap)
+        try:
+            res = []
+            for it in range(6):
+                x_dec = dev_bf16(W.normal_bf16(np.random.default_rng(it), (M, 1024)))
+                x_pre = dev_bf16(W.normal_bf16(np.random.default_rng(100 + it), (300, 1024)))
+                res.append(_dependent_chain(x_dec, x_pre, wts))
+            torch.cuda.synchronize()
+            B.check_status()
+        finally:
+            B.set_launch_overlap(False)
+        runs.append(res)
+    for other in runs[1:]:
+        for a, b in zip(runs[0], other):
+            for ta, tb in zip(a, b):
+                assert torch.equal(ta.view(torch.uint8), tb.view(torch.uint8))
