@@ -74,17 +74,11 @@ struct Params {
   uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ int group_of(const Params& p, int n) {
-  int g = 0;
-#pragma unroll
-  for (int i = 0; i < 7; ++i) g += (i < p.G - 1 && n >= p.group_end[i]) ? 1 : 0;
-  return g;
-}
-
 template <bool FP4, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                      const __grid_constant__ CUtensorMap tmW, const Params p) {
+                      const __grid_constant__ CUtensorMap tmW,
+                      const __grid_constant__ CUtensorMap tmY, const Params p) {
   using L = Layout<PAIR>;
   constexpr int S_TMA = L::S_TMA, S_W = L::S_W, S_B = L::S_B, BK = L::BK, A_BYTES = L::A_BYTES;
   extern __shared__ uint8_t smem_raw[];
@@ -244,6 +238,15 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     float gam[8];  // every group's weight scale, loaded once
 #pragma unroll
     for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
+    int ge[7];     // group ends in registers (past the last group: none)
+#pragma unroll
+    for (int g = 0; g < 7; ++g) ge[g] = g < p.G - 1 ? p.group_end[g] : 0x7FFFFFFF;
+    auto grp = [&](int col) {
+      int g = 0;
+#pragma unroll
+      for (int i = 0; i < 7; ++i) g += col >= ge[i] ? 1 : 0;
+      return g;
+    };
     pdl_wait();  // row scales come from the previous kernel; y may still be read by it
     uint32_t tl = 0;
     for (int tile = cta_slot; tile < p.num_tiles; tile += cta_stride, ++tl) {
@@ -266,8 +269,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         if (p.out_mode == kOutBf16) {
           // y = acc * (xs[m] * gamma[group(n)]); one scale per 32-column chunk
           // unless the chunk straddles a group boundary
-          const int g0 = group_of(p, n);
-          const int g1 = group_of(p, min(n + 31, p.N - 1));
+          const int g0 = grp(n);
+          const int g1 = grp(min(n + 31, p.N - 1));
           float s0 = 0.f;
 #pragma unroll
           for (int g = 0; g < 8; ++g) s0 = (g == g0) ? gam[g] : s0;
@@ -289,7 +292,12 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             // (a dynamic loop, so the common path above is not predicated)
 #pragma unroll 1
             for (int g = g0; g <= g1; ++g) {
-              const int lo = g == 0 ? 0 : p.group_end[g - 1], hi = p.group_end[g];
+              int lo = 0, hi = 0x7FFFFFFF;
+#pragma unroll
+              for (int j = 0; j < 7; ++j) {
+                lo = (j == g - 1) ? ge[j] : lo;
+                hi = (j == g) ? ge[j] : hi;
+              }
               float t = 0.f;
 #pragma unroll
               for (int j = 0; j < 8; ++j) t = (j == g) ? gam[j] : t;
@@ -302,29 +310,22 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-          // stage the warp's 32 x 32 bf16 block (64 B per row, 16-byte units
-          // swizzled by row) and write it back as 64-byte row segments:
-          // store s covers rows 8s..8s+7, four lanes per row
+          // stage the warp's 32 x 32 bf16 block (64 B per row, 16-byte unit v
+          // of row r at v ^ ((r >> 1) & 3): the 64-byte swizzle of the output
+          // tensor map) and write it with one TMA store; rows past M and
+          // columns past N are clipped by the map
+          if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
+          __syncwarp();
 #pragma unroll
           for (int v = 0; v < 4; ++v)
             st_shared_v4(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4), w[4 * v], w[4 * v + 1],
                          w[4 * v + 2], w[4 * v + 3]);
+          fence_proxy_async_smem();
           __syncwarp();
-          const int rr = lane >> 2, u = lane & 3;
-          uint4 o[4];
-#pragma unroll
-          for (int s2 = 0; s2 < 4; ++s2) {
-            const int row = 8 * s2 + rr;
-            o[s2] = ld_shared_v4(stg + row * 64 + ((u ^ ((row >> 1) & 3)) << 4));
+          if (lane == 0) {
+            tma_store_2d(&tmY, stg, n, m0 + q * 32);
+            bulk_commit();
           }
-#pragma unroll
-          for (int s2 = 0; s2 < 4; ++s2) {
-            const int mm = m0 + q * 32 + 8 * s2 + rr;
-            if (mm < p.M && n + 8 * u < p.N)
-              *reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.out) +
-                                        static_cast<int64_t>(mm) * p.ldo + n + 8 * u) = o[s2];
-          }
-          __syncwarp();
         } else if (row_ok) {
           uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
 #pragma unroll
@@ -342,6 +343,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         else      mbar_arrive(&tempty[acc]);
       }
     }
+    if (lane == 0) bulk_wait_all();  // output stores complete before the CTA exits
   } else if (warp >= 8) {
     // ------------------------------------------------------------- unpack
     const int ut = threadIdx.x - 256;  // 0..255
@@ -423,8 +425,8 @@ static cudaError_t make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const v
 }
 
 template <bool FP4, bool PAIR>
-static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const gemm::Params& p,
-                            cudaStream_t s) {
+static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const CUtensorMap& tmY,
+                            const gemm::Params& p, cudaStream_t s) {
   using namespace gemm;
   auto kern = bitlinear_gemm_kernel<FP4, PAIR>;
   static bool attr_set = false;  // once per process (not during graph capture)
@@ -438,10 +440,10 @@ static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, cons
   if (PAIR) {
     const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
     return launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS),
-                         Layout<PAIR>::SMEM_BYTES, s, 2u, tmA, tmW, p);
+                         Layout<PAIR>::SMEM_BYTES, s, 2u, tmA, tmW, tmY, p);
   }
   return launch_kernel(kern, dim3(static_cast<unsigned>(p.num_tiles < sms ? p.num_tiles : sms)),
-                       dim3(THREADS), Layout<PAIR>::SMEM_BYTES, s, 0u, tmA, tmW, p);
+                       dim3(THREADS), Layout<PAIR>::SMEM_BYTES, s, 0u, tmA, tmW, tmY, p);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why) {
@@ -451,7 +453,7 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   const bool pair = a.M > BM && a.K % 128 == 0;
   const int brows = pair ? BN / 2 : BN;
   const int BK = pair ? Layout<true>::BK : Layout<false>::BK;
-  CUtensorMap tmA, tmW;
+  CUtensorMap tmA, tmW, tmY;
   cudaError_t e;
   const CUtensorMapDataType adt = fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t row_bytes = fp4 ? a.K / 2 : a.K;
@@ -469,6 +471,14 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   e = make_map_2d(&tmW, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.Wp, a.K / 4, a.N, a.K / 4, BK / 4, brows,
                   CU_TENSOR_MAP_SWIZZLE_NONE, why);
   if (e != cudaSuccess) return e;
+  if (a.out_mode == kOutBf16) {
+    // bf16 Y [M x ldo], written by 32 x 32 TMA stores from 64-byte-swizzled staging
+    e = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.ldo * 2, 32, 32,
+                    CU_TENSOR_MAP_SWIZZLE_64B, why);
+    if (e != cudaSuccess) return e;
+  } else {
+    tmY = tmA;  // not used by the raw-accumulator epilogue
+  }
 
   Params p{};
   p.M = static_cast<int>(a.M);
@@ -489,8 +499,8 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
 
-  if (fp4) return pair ? launch_t<true, true>(tmA, tmW, p, s) : launch_t<true, false>(tmA, tmW, p, s);
-  return pair ? launch_t<false, true>(tmA, tmW, p, s) : launch_t<false, false>(tmA, tmW, p, s);
+  if (fp4) return pair ? launch_t<true, true>(tmA, tmW, tmY, p, s) : launch_t<true, false>(tmA, tmW, tmY, p, s);
+  return pair ? launch_t<false, true>(tmA, tmW, tmY, p, s) : launch_t<false, false>(tmA, tmW, tmY, p, s);
 }
 
 }  // namespace blt
