@@ -324,3 +324,81 @@ def test_launch_overlap_dependent_chain(M):
         for a, b in zip(runs[0], other):
             for ta, tb in zip(a, b):
                 assert torch.equal(ta.view(torch.uint8), tb.view(torch.uint8))
+
+
+# ---------------------------------------------- the bench's workloads, full size
+# Every kernel runs on the whole workload in the bench's launch configuration;
+# the oracle checks a seeded sample of token rows (each output row depends on
+# its own input row only) plus the full quantiser output where that is cheap.
+def _sample_rows(M, n, seed):
+    return np.sort(np.random.default_rng(seed).choice(M, n, replace=False))
+
+
+def _device_weights(proj):
+    Wp, gamma = B.ternarize_pack(proj.W, proj.group_ends)
+    return torch.from_numpy(Wp).to(DEV), torch.from_numpy(gamma).to(DEV)
+
+
+@pytest.mark.parametrize("mode", [O.MODE_INT4, O.MODE_FP4])
+def test_prefill_workload_full_size(mode):
+    """X [2048 x 2048] (1% outlier channels) through q|k|v [2048 x 6144] and
+    gate|up [2048 x 11264], as the bench's step runs them."""
+    d = W.input_projection_prefill(seed=1)
+    q, xs = B.quant_act(dev_bf16(d["x"]), mode)
+    q_o, xs_o = O.quant_act(d["x"], mode)
+    assert np.array_equal(host(q), q_o) and np.array_equal(host(xs), xs_o)
+    rows = _sample_rows(2048, 48, 11 + mode)
+    for proj in d["projs"]:
+        Wp, g = _device_weights(proj)
+        Wt, gamma = O.ternarize(proj.W, proj.group_ends)
+        if mode == O.MODE_FP4:
+            y = B.gemm_w2fp4(q, xs, Wp, g, proj.group_ends)
+            _, y_o = O.bitlinear_fp4(q_o[rows], xs_o[rows], Wt, gamma, proj.group_ends)
+        else:
+            y = B.gemm_w2a4(q, xs, Wp, g, proj.group_ends)
+            _, y_o = O.bitlinear_int(q_o[rows], xs_o[rows], Wt, gamma, proj.group_ends)
+        B.check_status()
+        assert_bf16_close(bits(y)[rows], y_o)
+
+
+def test_o_proj_workload_full_size():
+    """Top-k 50% + INT8 of X [4096 x 4096] (Student-t) and the o_proj GEMM."""
+    d = W.o_proj_sparse()
+    q, xs, _ = B.topk_sparsify_i8(dev_bf16(d["x"]))
+    rows = _sample_rows(4096, 48, 21)
+    q_o, xs_o, _ = O.topk_sparsify_i8(d["x"][rows])
+    assert np.array_equal(host(q)[rows], q_o) and np.array_equal(host(xs)[rows], xs_o)
+    Wp, g = _device_weights(d["proj"])
+    y = B.gemm_w2a8(q, xs, Wp, g, d["proj"].group_ends)
+    B.check_status()
+    Wt, gamma = O.ternarize(d["proj"].W, d["proj"].group_ends)
+    _, y_o = O.bitlinear_int(q_o, xs_o, Wt, gamma, d["proj"].group_ends)
+    assert_bf16_close(bits(y)[rows], y_o)
+
+
+def test_down_proj_workload_full_size():
+    """ReLU^2(gate) * up + INT8 of [4096 x 11008] and the down_proj GEMM."""
+    d = W.down_proj_relu2()
+    q, xs = B.quant_act(dev_bf16(d["gate"]), O.MODE_INT8, up=dev_bf16(d["up"]))
+    rows = _sample_rows(4096, 32, 31)
+    q_o, xs_o = O.quant_act(d["gate"][rows], O.MODE_INT8, up_bits=d["up"][rows])
+    assert np.array_equal(host(q)[rows], q_o) and np.array_equal(host(xs)[rows], xs_o)
+    Wp, g = _device_weights(d["proj"])
+    y = B.gemm_w2a8(q, xs, Wp, g, d["proj"].group_ends)
+    B.check_status()
+    Wt, gamma = O.ternarize(d["proj"].W, d["proj"].group_ends)
+    _, y_o = O.bitlinear_int(q_o, xs_o, Wt, gamma, d["proj"].group_ends)
+    assert_bf16_close(bits(y)[rows], y_o)
+
+
+def test_kv_workload_full_size():
+    """K and V caches [4096 x 32 x 128] with the bos token at 4 bits."""
+    d = W.decode_layer(batch=1, make_weights=False)
+    keep = torch.tensor([0], dtype=torch.int32, device=DEV)
+    for name in ("k_cache", "v_cache"):
+        kv = d[name]
+        c3, c4, sc = B.kv_quant_3bit(dev_bf16(kv), keep)
+        c3o, c4o, sco = O.kv_quant_3bit(kv, (0,))
+        assert np.array_equal(host(c3), c3o)
+        assert np.array_equal(host(c4), c4o)
+        assert np.array_equal(host(sc), sco)
