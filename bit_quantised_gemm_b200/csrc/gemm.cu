@@ -44,7 +44,7 @@ struct Layout {
   static constexpr int BK = PAIR ? 256 : 128;       // k-block depth in elements
   static constexpr int KSUB = BK / 128;             // 128-deep swizzled chunks per k-block
   static constexpr int S_TMA = PAIR ? 4 : 5;        // activation ring
-  static constexpr int S_W = PAIR ? 3 : 4;          // packed-weight ring
+  static constexpr int S_W = PAIR ? 2 : 4;          // packed-weight ring
   static constexpr int S_B = PAIR ? 2 : 3;          // unpacked-weight ring
   static constexpr int BROWS = PAIR ? BN / 2 : BN;  // weight rows staged per CTA
   static constexpr int A_BYTES = KSUB * SUB;
@@ -53,8 +53,8 @@ struct Layout {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + S_TMA * A_BYTES;
   static constexpr int OFF_WP = OFF_B + S_B * B_BYTES;
-  static constexpr int OFF_STG = OFF_WP + S_W * WP_BYTES;  // epilogue staging, 2 KB per warp
-  static constexpr int OFF_BAR = OFF_STG + 4 * 2048;
+  static constexpr int OFF_STG = OFF_WP + S_W * WP_BYTES;  // epilogue staging, 4 KB per warp
+  static constexpr int OFF_BAR = OFF_STG + 4 * 4096;
   static constexpr int N_BARS = 2 * S_TMA + 2 * S_W + 2 * S_B + 2 * 2 + 1;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
@@ -234,7 +234,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // ----------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quadrant
     const uint32_t tempty_addr0 = lead(&tempty[0]);
-    const uint32_t stg = smem_u32(smem + L::OFF_STG) + q * 2048;  // this warp's staging block
+    const uint32_t stg = smem_u32(smem + L::OFF_STG) + q * 4096;  // this warp's staging block
     float gam[8];  // every group's weight scale, loaded once
 #pragma unroll
     for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
@@ -260,33 +260,33 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       if (!mbar_wait(&tfull[acc], aph, tmo, s_abort)) { fail(); break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        const int n = n0 + c * 32;
+      for (int c = 0; c < BN / 64; ++c) {
+        const int n = n0 + c * 64;
         if (n >= p.N) break;  // warp-uniform
-        uint32_t r[32];
-        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 32, r);
+        uint32_t r[64];
+        tmem_ld64(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 64, r);
         tmem_ld_wait();
         if (p.out_mode == kOutBf16) {
-          // y = acc * (xs[m] * gamma[group(n)]); one scale per 32-column chunk
+          // y = acc * (xs[m] * gamma[group(n)]); one scale per 64-column chunk
           // unless the chunk straddles a group boundary
           const int g0 = grp(n);
-          const int g1 = grp(min(n + 31, p.N - 1));
+          const int g1 = grp(min(n + 63, p.N - 1));
           float s0 = 0.f;
 #pragma unroll
           for (int g = 0; g < 8; ++g) s0 = (g == g0) ? gam[g] : s0;
           s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
-          float f[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
+          for (int i = 0; i < 64; ++i) {
             // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
             // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
             // (1.5 * 2^23 + acc) - 1.5 * 2^23
-            f[i] = FP4 ? __uint_as_float(r[i])
-                       : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
+            const float f = FP4 ? __uint_as_float(r[i])
+                                : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
+            r[i] = __float_as_uint(f);
           }
           if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
 #pragma unroll
-            for (int i = 0; i < 32; ++i) f[i] = __fmul_rn(f[i], s0);
+            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), s0));
           } else {
             // the chunk crosses group boundaries: one pass per group touched
             // (a dynamic loop, so the common path above is not predicated)
@@ -303,23 +303,24 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               for (int j = 0; j < 8; ++j) t = (j == g) ? gam[j] : t;
               const float sg = __fmul_rn(xs_m, t);
 #pragma unroll
-              for (int i = 0; i < 32; ++i)
-                f[i] = (n + i >= lo && n + i < hi) ? __fmul_rn(f[i], sg) : f[i];
+              for (int i = 0; i < 64; ++i)
+                r[i] = (n + i >= lo && n + i < hi) ? __float_as_uint(__fmul_rn(__uint_as_float(r[i]), sg))
+                                                   : r[i];
             }
           }
-          uint32_t w[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(f[2 * i], f[2 * i + 1]);
-          // stage the warp's 32 x 32 bf16 block (64 B per row, 16-byte unit v
-          // of row r at v ^ ((r >> 1) & 3): the 64-byte swizzle of the output
-          // tensor map) and write it with one TMA store; rows past M and
-          // columns past N are clipped by the map
+          // stage the warp's 32 x 64 bf16 block (128 B per row, 16-byte unit v
+          // of row r at v ^ (r & 7): the 128-byte swizzle of the output tensor
+          // map) and write it with one TMA store; rows past M and columns
+          // past N are clipped by the map
           if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
           __syncwarp();
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            st_shared_v4(stg + lane * 64 + ((v ^ ((lane >> 1) & 3)) << 4), w[4 * v], w[4 * v + 1],
-                         w[4 * v + 2], w[4 * v + 3]);
+          for (int v = 0; v < 8; ++v)
+            st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
           fence_proxy_async_smem();
           __syncwarp();
           if (lane == 0) {
@@ -329,7 +330,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         } else if (row_ok) {
           uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < 16; ++v) {
             if (n + 4 * v >= p.N) break;
             reinterpret_cast<uint4*>(orow)[v] =
                 make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
@@ -472,9 +473,9 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
                   CU_TENSOR_MAP_SWIZZLE_NONE, why);
   if (e != cudaSuccess) return e;
   if (a.out_mode == kOutBf16) {
-    // bf16 Y [M x ldo], written by 32 x 32 TMA stores from 64-byte-swizzled staging
-    e = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.ldo * 2, 32, 32,
-                    CU_TENSOR_MAP_SWIZZLE_64B, why);
+    // bf16 Y [M x ldo], written by 32 x 64 TMA stores from 128-byte-swizzled staging
+    e = make_map_2d(&tmY, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a.out, a.N, a.M, a.ldo * 2, 64, 32,
+                    CU_TENSOR_MAP_SWIZZLE_128B, why);
     if (e != cudaSuccess) return e;
   } else {
     tmY = tmA;  // not used by the raw-accumulator epilogue
