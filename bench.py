@@ -677,6 +677,33 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
         k = {n: time_calls(torch, stream, [(lambda n=n, r=r: gemv(n, r)) for r in range(R)], steps, warm)
              for n in names}
         gemv_ms = sum(k.values())
+        fused = {}
+        if batch <= 8:
+            # the quantisers inside the GEMVs (bitlinear_gemv_w2_quant): 5 launches per layer
+            fq = {"qkv": (x, None, B.MODE_INT4), "gate_up": (x, None, B.MODE_INT4),
+                  "down": (ga, up, B.MODE_INT8)}
+
+            def gemv_q(name, r):
+                xa, ua, mode = fq[name]
+                B.gemv_w2_quant(xa, mode, wdev[r][name][0], wdev[r][name][1], shapes[name][2], up=ua,
+                                y=ys[name])
+
+            def l_step_fused(ev, r):
+                gemv_q("qkv", r)
+                B.topk_sparsify_i8(xo, out=qo, xs=xso)
+                gemv("o", r)
+                gemv_q("gate_up", r)
+                gemv_q("down", r)
+            gs, es = graph_set(torch, stream, [(lambda ev, r=r: l_step_fused(ev, r)) for r in range(R)],
+                               (), 4, timed=False)
+            fms, _, _ = run_graphs(torch, stream, gs, es, (), steps, warm)
+            del gs
+            fk = {n: time_calls(torch, stream, [(lambda n=n, r=r: gemv_q(n, r)) for r in range(R)], steps, warm)
+                  for n in fq}
+            fused = {"layer_step_us_quantisers_fused": round(fms / steps * 1e3, 2),
+                     "fused_gemv_us": {n: round(v * 1e3, 2) for n, v in fk.items()},
+                     "fused_note": "q|k|v, gate|up and down quantise their bf16 inputs inside the GEMV "
+                                   "(bitlinear_gemv_w2_quant); o keeps the separate top-k launch"}
         per = {n: {"us": round(k[n] * 1e3, 2), "GBps": round(K_ * N_ // 4 / k[n] / 1e6, 1)}
                for n, (K_, N_, _) in shapes.items()}
         dec[f"batch{batch}"] = {
@@ -686,7 +713,7 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
             "weight_GBps": round(wbytes / gemv_ms / 1e6, 1),
             "weight_frac_hbm": round(wbytes / gemv_ms / 1e6 / hbm, 4),
             "layer_weight_GBps_incl_quantisers": round(wbytes / (ms / steps) / 1e6, 1),
-            "per_projection": per}
+            "per_projection": per, **fused}
     out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=7,
                                        gemv_launches="qkv (fused, 3 groups), o, gate_up (fused, 2 groups), down",
                                        **dec)

@@ -48,6 +48,8 @@ _SIGS = {
     "bitlinear_gemm_w2a8_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
     "bitlinear_gemm_w2fp4_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
     "bitlinear_gemv_w2": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
+    "bitlinear_gemv_w2_quant": ([_P, _P, _I64, _INT, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P],
+                                _INT),
     "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
     "bitlinear_check_status": ([_P, _P], _INT),
     "bitlinear_debug_wait_timeout": ([_P, _I64, _P], _INT),
@@ -213,6 +215,25 @@ def gemm_w2fp4(xf4, xs, Wp, gamma, group_ends, y=None, status=None, stream=None)
 def gemv_w2(xq, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
     """Decode-time variant of gemm_w2a8 for 1..64 tokens."""
     return _gemm("bitlinear_gemv_w2", xq, xs, Wp, gamma, group_ends, xq.shape[1], y, status, stream)
+
+
+def gemv_w2_quant(x, mode, Wp, gamma, group_ends, up=None, y=None, status=None, stream=None):
+    """Decode-time BitLinear on bf16 activations (1..8 tokens): the per-token
+    INT8 / INT4 quantiser (ReLU^2-gated by `up` when given) runs inside the GEMV."""
+    _require_cuda(x, up, Wp, gamma)
+    if x.dim() != 2 or x.stride(1) != 1 or (up is not None and up.stride() != x.stride()):
+        raise ValueError("x (and up) must be row-major [M x K] with the same row stride")
+    M, K = x.shape
+    N = Wp.shape[0]
+    ge = np.ascontiguousarray(group_ends, dtype=np.int64)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    if status is None:
+        status = status_buffer(x.device)
+    _check(lib().bitlinear_gemv_w2_quant(_ptr(x), _ptr(up), x.stride(0), int(mode), _ptr(Wp), _ptr(gamma),
+                                         _ptr(ge), len(ge), M, N, K, _ptr(y), y.stride(0), _ptr(status),
+                                         _stream(stream)))
+    return y
 
 
 def gemm_w2a8_acc(xq, Wp, status=None, stream=None):

@@ -131,7 +131,7 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 101; }
+int bitlinear_version(void) { return 102; }
 
 int bitlinear_set_launch_overlap(int enable) {
   g_overlap.store(enable != 0);
@@ -298,6 +298,32 @@ int bitlinear_gemv_w2(const int8_t* xq, const float* xs, const uint8_t* Wp, cons
   const char* why = nullptr;
   cudaError_t e = blt::launch_gemv(a, stream, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2", why);
+}
+
+int bitlinear_gemv_w2_quant(const uint16_t* x, const uint16_t* up, int64_t ldx, int mode,
+                            const uint8_t* Wp, const float* gamma, const int64_t* group_ends, int G,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, int64_t ldy,
+                            int* dev_status, bitlinear_stream_t stream) {
+  blt::GemmArgs a{};
+  if (mode != BITLINEAR_MODE_INT8 && mode != BITLINEAR_MODE_INT4)
+    return fail(BITLINEAR_ERR_INVALID_ARG, "gemv_w2_quant: mode must be INT8 or INT4");
+  if (M > blt::kGemvDp4aMaxTokens)
+    return fail(BITLINEAR_ERR_UNSUPPORTED, "gemv_w2_quant: M=%lld above %d", (long long)M, blt::kGemvDp4aMaxTokens);
+  if (K % 128 != 0 || N % 128 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "gemv_w2_quant: K and N must be multiples of 128");
+  // the codes pointer checks apply to x; xs is not used (the kernel computes it)
+  const int rc = check_gemm("gemv_w2_quant", x, x, Wp, gamma, group_ends, G, M, N, K, y, ldy, true, &a);
+  if (rc != BITLINEAR_OK) return rc;
+  if (M == 0) return ok();
+  if (ldx < K || ldx % 8 != 0) return fail(BITLINEAR_ERR_INVALID_ARG, "gemv_w2_quant: ldx must be >= K and a multiple of 8");
+  if (up && !aligned16(up)) return fail(BITLINEAR_ERR_ALIGNMENT, "gemv_w2_quant: up must be 16-byte aligned");
+  if (!blt::gemv_dp4a_supported(M, K))
+    return fail(BITLINEAR_ERR_UNSUPPORTED, "gemv_w2_quant: K=%lld too large for %lld tokens", (long long)K, (long long)M);
+  a.out = y;
+  a.ldo = ldy;
+  a.out_mode = blt::kOutBf16;
+  a.status = dev_status;
+  cudaError_t e = blt::launch_gemv_dp4a_quant(a, x, up, ldx, mode, stream);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2_quant");
 }
 
 int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int32_t* keep4_pos,

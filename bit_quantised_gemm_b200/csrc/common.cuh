@@ -21,6 +21,31 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
   f[6] = bf16lo(v.w); f[7] = bf16hi(v.w);
 }
 
+// Integer code of one activation: clamp(rne(h * inv), lo, hi), fp32 multiply.
+__device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi) {
+  return static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(h, inv)), lo), hi));
+}
+
+__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
+  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
+         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
+}
+
+// h of the activation quantisers: x, or the ReLU^2-gated product
+// (r * r) * up with r = max(x, 0), both multiplies in fp32.
+__device__ __forceinline__ void act_vals8(const uint4& xv, const uint4& uv, bool relu2, float (&h)[8]) {
+  bf16x8_to_f32(xv, h);
+  if (relu2) {
+    float u[8];
+    bf16x8_to_f32(uv, u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float r = h[i] > 0.f ? h[i] : 0.f;
+      h[i] = __fmul_rn(__fmul_rn(r, r), u[i]);
+    }
+  }
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&h);

@@ -47,8 +47,12 @@ constexpr int SMEM_LIMIT = 232448;
 struct Params {
   int M, N, K;
   int n_items;
-  const int8_t* xq;
+  const int8_t* xq;     // activation codes [M x K] (codes given)
   const float* xs;
+  const uint16_t* x;    // bf16 activations [M x ldx] (quantised here)
+  const uint16_t* up;   // nullable: ReLU^2-gated product with x as the gate
+  int64_t ldx;
+  float Q;              // 127 (INT8) or 7 (INT4)
   const uint8_t* Wp;
   const float* gamma;
   int G;
@@ -159,7 +163,16 @@ __device__ __forceinline__ int combine(const int (&a)[NACC]) {
   else return a[0] + (a[1] >> 4);
 }
 
-template <int MT, int RW>
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
+  return v;
+}
+
+// FUSED: the kernel quantises the bf16 activations itself (per-token absmax,
+// INT8 / INT4, optionally of the ReLU^2-gated product), redundantly in every
+// CTA, instead of reading codes written by a separate quantiser launch.
+template <int MT, int RW, bool FUSED>
 __global__ void __launch_bounds__(MAX_WARPS * 32, 1)
 bitlinear_gemv_dp4a_kernel(const Params p) {
   constexpr int NACC = MT <= 2 ? 4 : 2;
@@ -206,37 +219,75 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
   float gam[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) gam[i] = i < p.G ? __ldg(p.gamma + i) : 0.f;
-  pdl_trigger();
-  pdl_wait();  // activation codes and scales come from the previous kernel
-  if (threadIdx.x == 0) {  // the codes are one contiguous M x K block
-    const uint32_t xbytes = static_cast<uint32_t>(p.M * K);
-    mbar_arrive_expect_tx(xbar, xbytes);
-    bulk_load(smem_u32(xsm), p.xq, xbytes, xbar);
-  }
   float xsc[MT];
+  bool x_ok = true;
+  pdl_trigger();
+  if constexpr (FUSED) {
+    pdl_wait();  // the bf16 activations come from the previous kernel
+    float* red = reinterpret_cast<float*>(xsum + MT);  // [nwarps][MT] partial maxima
+    if (threadIdx.x < MT) xsum[threadIdx.x] = 0;
+    for (int i = p.M * K / 16 + threadIdx.x; i < MT * K / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(xsm)[i] = make_uint4(0u, 0u, 0u, 0u);  // tokens M.. are zero
+    const int G16 = K >> 4;  // 16-element groups per row
+    const bool relu2 = p.up != nullptr;
+    auto load16 = [&](int t, int g, float (&h)[16]) {
+      const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * p.ldx) + 2 * g;
+      const uint4* ur = relu2 ? reinterpret_cast<const uint4*>(p.up + static_cast<int64_t>(t) * p.ldx) + 2 * g : xr;
+      float a[8], b[8];
+      act_vals8(__ldg(xr), relu2 ? __ldg(ur) : make_uint4(0u, 0u, 0u, 0u), relu2, a);
+      act_vals8(__ldg(xr + 1), relu2 ? __ldg(ur + 1) : make_uint4(0u, 0u, 0u, 0u), relu2, b);
 #pragma unroll
-  for (int t = 0; t < MT; ++t) xsc[t] = t < p.M ? __ldg(p.xs + t) : 0.f;
-  if (threadIdx.x < MT) xsum[threadIdx.x] = 0;
-  // tokens p.M .. MT-1 are zero codes
-  for (int i = p.M * K / 16 + threadIdx.x; i < MT * K / 16; i += blockDim.x)
-    reinterpret_cast<uint4*>(xsm)[i] = make_uint4(0u, 0u, 0u, 0u);
-  __syncthreads();
-
-  // Regroup the codes in place and take their row sums.
-  const bool x_ok = mbar_wait(xbar, 0, p.timeout_ns, nullptr);
-  if (x_ok) {
-    const int groups = p.M * K / 16;
+      for (int i = 0; i < 8; ++i) { h[i] = a[i]; h[8 + i] = b[i]; }
+    };
+    // pass 1: absmax of every token row
+    float am[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) am[t] = 0.f;
+    for (int i = threadIdx.x; i < p.M * G16; i += blockDim.x) {
+      const int t = i / G16, g = i - t * G16;
+      float h[16];
+      load16(t, g, h);
+      float mx = 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) mx = fmaxf(mx, fabsf(h[j]));
+#pragma unroll
+      for (int u = 0; u < MT; ++u) am[u] = (u == t) ? fmaxf(am[u], mx) : am[u];
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      am[t] = warp_max_f(am[t]);
+      if (lane == 0) red[warp * MT + t] = am[t];
+    }
+    __syncthreads();
+    float inv[MT];
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      float a = 0.f;
+      for (int w = 0; w < nwarps; ++w) a = fmaxf(a, red[w * MT + t]);
+      a = fmaxf(a, kEps);
+      inv[t] = __fdiv_rn(p.Q, a);
+      xsc[t] = t < p.M ? __fdiv_rn(a, p.Q) : 0.f;
+    }
+    // pass 2: the codes, regrouped into shared memory, and their row sums
     int part[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) part[t] = 0;
-    for (int i = threadIdx.x; i < groups; i += blockDim.x) {
-      uint4* q = reinterpret_cast<uint4*>(xsm) + i;
-      const uint4 v = *q;
-      const int t = i / (K / 16);
+    for (int i = threadIdx.x; i < p.M * G16; i += blockDim.x) {
+      const int t = i / G16, g = i - t * G16;
+      float h[16];
+      load16(t, g, h);
+      float iv = 0.f;
+#pragma unroll
+      for (int u = 0; u < MT; ++u) iv = (u == t) ? inv[u] : iv;
+      int q[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) q[j] = quant_code(h[j], iv, -p.Q - 1.f, p.Q);
+      const uint4 v = make_uint4(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]),
+                                 pack_s8x4(q[8], q[9], q[10], q[11]), pack_s8x4(q[12], q[13], q[14], q[15]));
       const int bs = byte_sum16(v);
 #pragma unroll
       for (int u = 0; u < MT; ++u) part[u] += (u == t) ? bs : 0;
-      *q = regroup16(v);
+      *reinterpret_cast<uint4*>(xsm + t * K + 16 * g) = regroup16(v);
     }
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
@@ -244,8 +295,47 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
       for (int o = 16; o >= 1; o >>= 1) part[t] += __shfl_xor_sync(0xFFFFFFFFu, part[t], o);
       if (lane == 0 && part[t] != 0) atomicAdd(&xsum[t], part[t]);
     }
+    __syncthreads();
+  } else {
+    pdl_wait();  // activation codes and scales come from the previous kernel
+    if (threadIdx.x == 0) {  // the codes are one contiguous M x K block
+      const uint32_t xbytes = static_cast<uint32_t>(p.M * K);
+      mbar_arrive_expect_tx(xbar, xbytes);
+      bulk_load(smem_u32(xsm), p.xq, xbytes, xbar);
+    }
+#pragma unroll
+    for (int t = 0; t < MT; ++t) xsc[t] = t < p.M ? __ldg(p.xs + t) : 0.f;
+    if (threadIdx.x < MT) xsum[threadIdx.x] = 0;
+    // tokens p.M .. MT-1 are zero codes
+    for (int i = p.M * K / 16 + threadIdx.x; i < MT * K / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(xsm)[i] = make_uint4(0u, 0u, 0u, 0u);
+    __syncthreads();
+
+    // Regroup the codes in place and take their row sums.
+    x_ok = mbar_wait(xbar, 0, p.timeout_ns, nullptr);
+    if (x_ok) {
+      const int groups = p.M * K / 16;
+      int part[MT];
+#pragma unroll
+      for (int t = 0; t < MT; ++t) part[t] = 0;
+      for (int i = threadIdx.x; i < groups; i += blockDim.x) {
+        uint4* q = reinterpret_cast<uint4*>(xsm) + i;
+        const uint4 v = *q;
+        const int t = i / (K / 16);
+        const int bs = byte_sum16(v);
+#pragma unroll
+        for (int u = 0; u < MT; ++u) part[u] += (u == t) ? bs : 0;
+        *q = regroup16(v);
+      }
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) part[t] += __shfl_xor_sync(0xFFFFFFFFu, part[t], o);
+        if (lane == 0 && part[t] != 0) atomicAdd(&xsum[t], part[t]);
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
   int xsm_sum[MT];
 #pragma unroll
   for (int t = 0; t < MT; ++t) xsm_sum[t] = xsum[t];
@@ -328,7 +418,7 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
     if (lane == 0)
       for (int q = s; q < min(s + SW, n_mine); ++q)
         mbar_wait(my_bar + (q % SW), (q / SW) & 1, p.timeout_ns, nullptr);
-    if (threadIdx.x == 0 && !x_ok) mbar_wait(xbar, 0, p.timeout_ns, nullptr);
+    if (!FUSED && threadIdx.x == 0 && !x_ok) mbar_wait(xbar, 0, p.timeout_ns, nullptr);
     __syncwarp();
   }
 }
@@ -337,7 +427,7 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 
 static size_t dp4a_smem_bytes(int mt, int rw, int64_t K, int warps) {
   return size_t(mt) * K + size_t(warps) * gemv_cc::SW * rw * (K / 4) +
-         size_t(warps) * gemv_cc::SW * 8 + 8 + 8 * 4;
+         size_t(warps) * gemv_cc::SW * 8 + 8 + 8 * 4 + size_t(gemv_cc::MAX_WARPS) * mt * 4;
 }
 
 static int dp4a_tokens(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 4 ? 4 : 8; }
@@ -355,14 +445,14 @@ bool gemv_dp4a_supported(int64_t M, int64_t K) {
   return dp4a_warps_fit(dp4a_tokens(M), 2, K) > 0;
 }
 
-template <int MT, int RW>
+template <int MT, int RW, bool FUSED>
 static cudaError_t launch_mt(gemv_cc::Params p, cudaStream_t s) {
   p.n_items = (p.N + RW - 1) / RW;
   const int grid = std::min(num_sms(), p.n_items);
   int warps = (p.n_items + grid - 1) / grid;
   warps = std::min(warps, dp4a_warps_fit(MT, RW, p.K));
   const size_t smem = dp4a_smem_bytes(MT, RW, p.K, warps);
-  auto kern = gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW>;
+  auto kern = gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -371,17 +461,27 @@ static cudaError_t launch_mt(gemv_cc::Params p, cudaStream_t s) {
 
 // Items of 4 output features when there are enough of them to give every
 // SM a full complement of warps (and the ring fits), else of 2.
-template <int MT>
+template <int MT, bool FUSED>
 static cudaError_t launch_pick_rows(const gemv_cc::Params& p, cudaStream_t s) {
   if constexpr (MT <= 4) {  // eight tokens: 2 rows (registers)
     if (int64_t(p.N) >= int64_t(4) * gemv_cc::MAX_WARPS * num_sms() &&
         dp4a_warps_fit(MT, 4, p.K) == gemv_cc::MAX_WARPS)
-      return launch_mt<MT, 4>(p, s);
+      return launch_mt<MT, 4, FUSED>(p, s);
   }
-  return launch_mt<MT, 2>(p, s);
+  return launch_mt<MT, 2, FUSED>(p, s);
 }
 
-cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s) {
+template <bool FUSED>
+static cudaError_t launch_by_tokens(const gemv_cc::Params& p, cudaStream_t s) {
+  switch (dp4a_tokens(p.M)) {
+    case 1: return launch_pick_rows<1, FUSED>(p, s);
+    case 2: return launch_pick_rows<2, FUSED>(p, s);
+    case 4: return launch_pick_rows<4, FUSED>(p, s);
+    default: return launch_pick_rows<8, FUSED>(p, s);
+  }
+}
+
+static gemv_cc::Params dp4a_params(const GemmArgs& a) {
   gemv_cc::Params p{};
   p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
@@ -396,12 +496,21 @@ cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s) {
   p.ldy = a.ldo;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
-  switch (dp4a_tokens(a.M)) {
-    case 1: return launch_pick_rows<1>(p, s);
-    case 2: return launch_pick_rows<2>(p, s);
-    case 4: return launch_pick_rows<4>(p, s);
-    default: return launch_pick_rows<8>(p, s);
-  }
+  return p;
+}
+
+cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s) {
+  return launch_by_tokens<false>(dp4a_params(a), s);
+}
+
+cudaError_t launch_gemv_dp4a_quant(const GemmArgs& a, const uint16_t* x, const uint16_t* up,
+                                   int64_t ldx, int mode, cudaStream_t s) {
+  gemv_cc::Params p = dp4a_params(a);
+  p.x = x;
+  p.up = up;
+  p.ldx = ldx;
+  p.Q = mode == BITLINEAR_MODE_INT8 ? 127.f : 7.f;
+  return launch_by_tokens<true>(p, s);
 }
 
 }  // namespace blt

@@ -44,6 +44,10 @@ cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why);
 constexpr int kGemvDp4aMaxTokens = 8;
 bool gemv_dp4a_supported(int64_t M, int64_t K);
 cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s);
+// The same with the per-token quantiser (INT8 / INT4, optional ReLU^2 gate)
+// done inside the GEMV on bf16 activations x [M x ldx].
+cudaError_t launch_gemv_dp4a_quant(const GemmArgs& a, const uint16_t* x, const uint16_t* up,
+                                   int64_t ldx, int mode, cudaStream_t s);
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s);
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once at run time.

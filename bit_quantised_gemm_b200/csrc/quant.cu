@@ -55,15 +55,6 @@ __device__ __forceinline__ uint32_t block_scan_256(uint32_t v, uint32_t* sums /*
   return v;
 }
 
-__device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi) {
-  return static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(h, inv)), lo), hi));
-}
-
-__device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
-  return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
-         ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);
-}
-
 // 8 fp32 -> 8 e2m1 nibbles (even index low), round to nearest even, satfinite.
 __device__ __forceinline__ uint32_t cvt_e2m1x8(const float (&v)[8]) {
   uint32_t out;

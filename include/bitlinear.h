@@ -159,6 +159,25 @@ int bitlinear_gemv_w2(const int8_t* xq, const float* xs, const uint8_t* Wp, cons
                       uint16_t* y, int64_t ldy, int* dev_status, bitlinear_stream_t stream);
 
 /*
+ * Decode-time BitLinear with the activation quantiser fused in: the same
+ * result, bit for bit, as bitlinear_quant_act(x, up, M, K, ldx, mode) followed
+ * by bitlinear_gemv_w2 on its codes ([R] "Метод": INT4 codes on the q/k/v and
+ * gate/up inputs, ReLU^2 gate then INT8 on the down_proj input; [A] abstract:
+ * 4-bit activations), without the codes ever reaching HBM: every CTA
+ * quantises the few token rows itself.
+ *   x, up   device bf16 [M x ldx]; up nullable (ReLU^2 gate when given)
+ *   mode    BITLINEAR_MODE_INT8 or BITLINEAR_MODE_INT4
+ *   other arguments as bitlinear_gemv_w2
+ * Requires 1 <= M <= 8 (BITLINEAR_ERR_UNSUPPORTED above), ldx >= K,
+ * ldx % 8 == 0, x and up 16-byte aligned, and the bitlinear_gemv_w2
+ * requirements.
+ */
+int bitlinear_gemv_w2_quant(const uint16_t* x, const uint16_t* up, int64_t ldx, int mode,
+                            const uint8_t* Wp, const float* gamma, const int64_t* group_ends, int G,
+                            int64_t M, int64_t N, int64_t K, uint16_t* y, int64_t ldy,
+                            int* dev_status, bitlinear_stream_t stream);
+
+/*
  * KV-cache quantiser ([R] "Эксперименты": 3-bit KV cache, the <bos> and
  * <eos> tokens kept at 4 bits). Per (token t, head h) over the head dim:
  *   a' = max(max_d |x|, 1e-5f); tokens listed in keep4_pos: Q = 7, codes in

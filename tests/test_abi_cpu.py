@@ -20,7 +20,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(_lib._SIGS)
-    assert B.version() == 101
+    assert B.version() == 102
 
 
 @pytest.mark.parametrize("K,N,groups,seed", [
@@ -86,6 +86,25 @@ def test_gemm_argument_errors(fn):
 def test_gemv_and_fp4_specific_limits():
     assert _gemm("bitlinear_gemv_w2", M=65) == _lib.ERR_INVALID_ARG
     assert _gemm("bitlinear_gemm_w2fp4", K=192) == _lib.ERR_INVALID_ARG  # K % 128
+
+
+def test_fused_gemv_argument_errors():
+    def call(**kw):
+        a = dict(x=FAKE, up=None, ldx=256, mode=1, Wp=FAKE, gamma=FAKE, ge=ge1.ctypes.data, G=1,
+                 M=4, N=256, K=256, y=FAKE, ldy=256)
+        a.update(kw)
+        return B.lib().bitlinear_gemv_w2_quant(a["x"], a["up"], a["ldx"], a["mode"], a["Wp"], a["gamma"],
+                                               a["ge"], a["G"], a["M"], a["N"], a["K"], a["y"], a["ldy"],
+                                               None, None)
+    assert call(mode=2) == _lib.ERR_INVALID_ARG        # FP4 is not a GEMV code kind
+    assert call(M=9) == _lib.ERR_UNSUPPORTED            # more tokens: quantiser + GEMV
+    assert call(K=192) == _lib.ERR_INVALID_ARG          # K % 128
+    assert call(ldx=128) == _lib.ERR_INVALID_ARG        # ldx < K
+    assert call(ldx=260) == _lib.ERR_INVALID_ARG        # ldx % 8
+    assert call(x=FAKE + 2) == _lib.ERR_ALIGNMENT
+    assert call(up=FAKE + 2) == _lib.ERR_ALIGNMENT
+    assert call(x=None) == _lib.ERR_INVALID_ARG
+    assert call(M=0) == _lib.OK
 
 
 def test_quantiser_argument_errors():

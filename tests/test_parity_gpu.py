@@ -291,6 +291,8 @@ def _dependent_chain(x_dec, x_pre, wts):
     y = B.gemv_w2(q, xs, Wp2, g2, (1024,))
     q, xs = B.topk_sparsify_i8(y)[:2]
     outs.append(B.gemv_w2(q, xs, Wp3, g3, (1024,)))
+    if outs[-1].shape[0] <= 8:  # the fused quantiser + GEMV reads the previous output directly
+        outs.append(B.gemv_w2_quant(outs[-1], O.MODE_INT8, Wp1, g1, (1024,), up=outs[-1]))
     q, xs = B.quant_act(x_pre, O.MODE_INT4)
     y = B.gemm_w2a4(q, xs, Wp1, g1, (1024,))
     q, xs = B.topk_sparsify_i8(y)[:2]
@@ -402,3 +404,40 @@ def test_kv_workload_full_size():
         assert np.array_equal(host(c3), c3o)
         assert np.array_equal(host(c4), c4o)
         assert np.array_equal(host(sc), sco)
+
+
+@pytest.mark.parametrize("M", [1, 3, 8])
+@pytest.mark.parametrize("mode,relu2", [(O.MODE_INT4, False), (O.MODE_INT8, False), (O.MODE_INT8, True)])
+@pytest.mark.parametrize("N,K", [(4096, 4096), (4096, 11008), (128, 128)])
+def test_gemv_quant_fused(M, mode, relu2, N, K):
+    """The quantiser inside the GEMV gives the oracle's quantiser + BitLinear,
+    and the same bits as the two separate calls."""
+    rng = np.random.default_rng(M * 7 + K + mode)
+    x = W.outlier_bf16(rng, M, K)[0]
+    up = W.normal_bf16(rng, (M, K)) if relu2 else None
+    groups = (N // 2, N)
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, groups, 17)
+    xd = dev_bf16(x)
+    ud = dev_bf16(up) if relu2 else None
+    y = B.gemv_w2_quant(xd, mode, Wp, gamma_d, groups, up=ud)
+    B.check_status()
+    xq_o, xs_o = O.quant_act(x, mode, up_bits=up)
+    _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, groups)
+    assert_bf16_close(bits(y), y_o)
+    q, xs = B.quant_act(xd, mode, up=ud)
+    y2 = B.gemv_w2(q, xs, Wp, gamma_d, groups)
+    assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+def test_gemv_quant_fused_strided_rows():
+    """Rows with a stride above K (a view into a wider buffer)."""
+    M, K, N = 5, 4096, 1024
+    rng = np.random.default_rng(5)
+    wide = W.normal_bf16(rng, (M, K + 64))
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, (N,), 18)
+    xd = dev_bf16(wide)[:, :K]
+    y = B.gemv_w2_quant(xd, O.MODE_INT4, Wp, gamma_d, (N,))
+    B.check_status()
+    xq_o, xs_o = O.quant_act(np.ascontiguousarray(wide[:, :K]), O.MODE_INT4)
+    _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, (N,))
+    assert_bf16_close(bits(y), y_o)
