@@ -55,6 +55,9 @@ CUDA library implements from its own code) are:
      3-bit stream (code d in bits [3d, 3d+3)); tokens listed in keep4_pos use
      Q = 7, clamp [-8, 7], stored as code + 8, two per byte, low nibble first;
      their 3-bit row is all zero bytes. scale = a' / Q.
+  C10 decode attention over that cache (the pages name only its storage
+     precision): softmax((q . k_t) / sqrt(D)) over every cached token t of
+     the query's head, weights applied to the dequantised v_t; fp64 here.
 
 Quantisation decisions are taken in fp32 (the precision of the kernels),
 because a float decides an integer there; everything else is fp64 or exact.
@@ -380,6 +383,33 @@ def kv_dequant(codes3, codes4, scale, keep4_pos, D):
         u4[:, 1::2] = codes4[j] >> 4
         out[t] = (u4 - 8) * scale[t][:, None]
     return out
+
+
+def kv_attention_f64(q_bits, k_store, v_store, keep4_pos):
+    """Decode attention over the C9 cache (the consumer of the 3-bit KV
+    quantiser; [R] "Эксперименты": 3-bit KV cache). The pages state only the
+    storage precision; the attention is the plain scaled dot-product one
+    (reading C10): for each query (b, h) and every cached token t of head h,
+      s_t = (q . k_t) / sqrt(D),  p = softmax_t(s),  o = sum_t p_t v_t
+    with k_t, v_t the dequantised cache rows (code * scale) and q the bf16
+    query. Everything in fp64.
+
+    q_bits: bf16 bits [B x H x D]; k_store, v_store: (codes3, codes4, scale)
+    as returned by kv_quant_3bit. Returns o as fp64 [B x H x D]."""
+    q = bf16_to_f32(q_bits).astype(np.float64)
+    D = q.shape[2]
+    k = kv_dequant(*k_store, keep4_pos, D)  # [T x H x D]
+    v = kv_dequant(*v_store, keep4_pos, D)
+    s = np.einsum("bhd,thd->bht", q, k) / math.sqrt(D)
+    s = s - s.max(axis=2, keepdims=True)
+    p = np.exp(s)
+    p = p / p.sum(axis=2, keepdims=True)
+    return np.einsum("bht,thd->bhd", p, v)
+
+
+def kv_attention_3bit(q_bits, k_store, v_store, keep4_pos):
+    """kv_attention_f64 rounded to bf16 (nearest even)."""
+    return f64_to_bf16(kv_attention_f64(q_bits, k_store, v_store, keep4_pos))
 
 
 def ceil_half(K: int) -> int:

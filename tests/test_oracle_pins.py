@@ -331,3 +331,68 @@ def test_kv_invariants_and_roundtrip():
     rest = [t for t in range(T) if t not in keep]
     assert u3[rest].min() >= 1 and u3[rest].max() <= 7   # codes in [-3, 3]
     assert np.all(c3[list(keep)] == 0)
+
+
+# ---------------------------------------------------------- C10 attention
+def _kv_store(rng, T, H, D, keep):
+    kv = W.normal_bf16(rng, (T, H, D))
+    return O.kv_quant_3bit(kv, keep), kv
+
+
+def test_attention_single_token_returns_its_value_row():
+    """One cached token: softmax weight 1, the output is that token's
+    dequantised value row (exactly, before the bf16 rounding)."""
+    rng = np.random.default_rng(40)
+    (ks, _), (vs, _) = _kv_store(rng, 1, 2, 64, (0,)), _kv_store(rng, 1, 2, 64, (0,))
+    q = W.normal_bf16(rng, (3, 2, 64))
+    o = O.kv_attention_f64(q, ks, vs, (0,))
+    v = O.kv_dequant(*vs, (0,), 64)
+    assert np.array_equal(o, np.broadcast_to(v[0], (3, 2, 64)))
+
+
+def test_attention_zero_query_is_the_mean_value():
+    rng = np.random.default_rng(41)
+    T, H, D = 37, 3, 128
+    ks, _ = _kv_store(rng, T, H, D, (0, 5))
+    vs, _ = _kv_store(rng, T, H, D, (0, 5))
+    q = np.zeros((1, H, D), dtype=np.uint16)  # +0.0 in bf16
+    o = O.kv_attention_f64(q, ks, vs, (0, 5))
+    v = O.kv_dequant(*vs, (0, 5), D)
+    assert np.allclose(o[0], v.mean(axis=0), rtol=1e-12, atol=1e-14)
+
+
+def test_attention_two_tokens_closed_form():
+    """Two tokens, one head: o = (e^a v0 + e^b v1) / (e^a + e^b) with a, b
+    the two scaled scores, written out with scalar math."""
+    rng = np.random.default_rng(42)
+    D = 64
+    ks, _ = _kv_store(rng, 2, 1, D, ())
+    vs, _ = _kv_store(rng, 2, 1, D, ())
+    q = W.normal_bf16(rng, (1, 1, D))
+    k = O.kv_dequant(*ks, (), D)[:, 0]
+    v = O.kv_dequant(*vs, (), D)[:, 0]
+    qf = O.bf16_to_f32(q)[0, 0].astype(np.float64)
+    a = sum(float(qf[d]) * float(k[0, d]) for d in range(D)) / math.sqrt(D)
+    b = sum(float(qf[d]) * float(k[1, d]) for d in range(D)) / math.sqrt(D)
+    ea, eb = math.exp(a - max(a, b)), math.exp(b - max(a, b))
+    want = [(ea * float(v[0, d]) + eb * float(v[1, d])) / (ea + eb) for d in range(D)]
+    o = O.kv_attention_f64(q, ks, vs, ())
+    assert np.allclose(o[0, 0], want, rtol=1e-12, atol=1e-14)
+
+
+def test_attention_token_order_invariance():
+    """Permuting the cached tokens (and the 4-bit list with them) leaves the
+    output unchanged."""
+    rng = np.random.default_rng(43)
+    T, H, D = 29, 2, 64
+    k_bits = W.normal_bf16(rng, (T, H, D))
+    v_bits = W.normal_bf16(rng, (T, H, D))
+    keep = (0, 11)
+    q = W.normal_bf16(rng, (2, H, D))
+    o1 = O.kv_attention_f64(q, O.kv_quant_3bit(k_bits, keep), O.kv_quant_3bit(v_bits, keep), keep)
+    perm = rng.permutation(T)
+    inv = np.argsort(perm)
+    keep2 = tuple(sorted(int(inv[t]) for t in keep))
+    o2 = O.kv_attention_f64(q, O.kv_quant_3bit(k_bits[perm], keep2), O.kv_quant_3bit(v_bits[perm], keep2),
+                            keep2)
+    assert np.allclose(o1, o2, rtol=1e-12, atol=1e-14)
