@@ -131,7 +131,7 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 102; }
+int bitlinear_version(void) { return 103; }
 
 int bitlinear_set_launch_overlap(int enable) {
   g_overlap.store(enable != 0);
@@ -341,6 +341,28 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
     return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: T * H * D / 8 must stay below 2^32");
   cudaError_t e = blt::launch_kv_quant(kv, T, H, D, keep4_pos, n_keep4, codes3, codes4, scale, stream);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_quant_3bit launch");
+}
+
+int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
+                      const uint8_t* k_codes3, const uint8_t* k_codes4, const float* k_scale,
+                      const uint8_t* v_codes3, const uint8_t* v_codes4, const float* v_scale,
+                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out,
+                      bitlinear_stream_t stream) {
+  if (B < 0 || H <= 0 || T <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: bad sizes");
+  if (D != 64 && D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: D must be 64, 128 or 256");
+  if (n_keep4 < 0 || n_keep4 > T || (n_keep4 > 0 && (!keep4_pos || !k_codes4 || !v_codes4)))
+    return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: bad 4-bit token list");
+  if (n_keep4 > 1024) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: at most 1024 tokens at 4 bits");
+  if (H > 65535 || (B + 7) / 8 > 65535 || T >= (1LL << 31) / H)
+    return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: sizes beyond the supported range");
+  if (B == 0) return ok();
+  if (!q || !k_codes3 || !k_scale || !v_codes3 || !v_scale || !out)
+    return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: null pointer");
+  if (!aligned16(q) || !aligned16(k_codes3) || !aligned16(v_codes3) || !aligned16(out))
+    return fail(BITLINEAR_ERR_ALIGNMENT, "kv_attention_3bit: q, codes and out must be 16-byte aligned");
+  cudaError_t e = blt::launch_kv_attention(q, B, H, D, T, k_codes3, k_codes4, k_scale, v_codes3,
+                                           v_codes4, v_scale, keep4_pos, n_keep4, out, stream);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "kv_attention_3bit launch");
 }
 
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream) {

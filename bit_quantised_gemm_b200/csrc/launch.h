@@ -12,6 +12,10 @@ cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, i
                              int64_t ldx, int mode, void* q, float* xs, cudaStream_t s);
 cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, int64_t k,
                            int8_t* q, float* xs, uint8_t* mask, cudaStream_t s);
+cudaError_t launch_kv_attention(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
+                                const uint8_t* k3, const uint8_t* k4, const float* ks,
+                                const uint8_t* v3, const uint8_t* v4, const float* vs,
+                                const int32_t* keep4, int64_t n4, uint16_t* out, cudaStream_t s);
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s);

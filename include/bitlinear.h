@@ -199,6 +199,28 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
                   int64_t n_keep4, uint8_t* codes3, uint8_t* codes4, float* scale,
                   bitlinear_stream_t stream);
 
+/*
+ * Decode attention over that cache ([R] "Эксперименты": the 3-bit KV cache
+ * with <bos>/<eos> at 4 bits is what attention reads at inference). For
+ * every query (b, h) and every cached token t < T of head h:
+ *   s_t = (q[b,h] . k[t,h]) / sqrt(D),  p = softmax_t(s),
+ *   out[b,h] = bf16_rne(sum_t p_t v[t,h])
+ * with k, v dequantised from the kv_quant_3bit storage ((code) * scale), in
+ * fp32 with an online softmax. Agrees with the fp64 result within one bf16
+ * ulp plus 2.5e-4 of the largest |v| (fp32 accumulation over T terms).
+ *   q          device bf16 [B x H x D]
+ *   k_*, v_*   codes3 / codes4 / scale of K and V as written by kv_quant_3bit
+ *              with the same keep4_pos list (codes4 nullable iff n_keep4 == 0)
+ *   keep4_pos  device int32 [n_keep4], strictly increasing, n_keep4 <= 1024
+ *   out        device bf16 [B x H x D]
+ * Requires D in {64, 128, 256}, T >= 1; B == 0 launches nothing.
+ */
+int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
+                      const uint8_t* k_codes3, const uint8_t* k_codes4, const float* k_scale,
+                      const uint8_t* v_codes3, const uint8_t* v_codes4, const float* v_scale,
+                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out,
+                      bitlinear_stream_t stream);
+
 /* Synchronise the stream and read *dev_status: BITLINEAR_OK, or
  * BITLINEAR_ERR_TIMEOUT if a kernel gave up a bounded wait. */
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream);

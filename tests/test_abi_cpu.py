@@ -20,7 +20,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(_lib._SIGS)
-    assert B.version() == 102
+    assert B.version() == 103
 
 
 @pytest.mark.parametrize("K,N,groups,seed", [
@@ -105,6 +105,23 @@ def test_fused_gemv_argument_errors():
     assert call(up=FAKE + 2) == _lib.ERR_ALIGNMENT
     assert call(x=None) == _lib.ERR_INVALID_ARG
     assert call(M=0) == _lib.OK
+
+
+def test_kv_attention_argument_errors():
+    L = B.lib()
+    def call(**kw):
+        a = dict(q=FAKE, B=2, H=4, D=128, T=64, k3=FAKE, k4=None, ks=FAKE, v3=FAKE, v4=None, vs=FAKE,
+                 keep=None, n4=0, out=FAKE)
+        a.update(kw)
+        return L.kv_attention_3bit(a["q"], a["B"], a["H"], a["D"], a["T"], a["k3"], a["k4"], a["ks"],
+                                   a["v3"], a["v4"], a["vs"], a["keep"], a["n4"], a["out"], None)
+    assert call(D=96) == _lib.ERR_UNSUPPORTED
+    assert call(T=0) == _lib.ERR_INVALID_ARG
+    assert call(n4=1) == _lib.ERR_INVALID_ARG               # no list / 4-bit rows
+    assert call(n4=65, keep=FAKE, k4=FAKE, v4=FAKE) == _lib.ERR_INVALID_ARG  # more than T
+    assert call(q=None) == _lib.ERR_INVALID_ARG
+    assert call(out=FAKE + 2) == _lib.ERR_ALIGNMENT
+    assert call(B=0) == _lib.OK
 
 
 def test_quantiser_argument_errors():

@@ -441,3 +441,57 @@ def test_gemv_quant_fused_strided_rows():
     xq_o, xs_o = O.quant_act(np.ascontiguousarray(wide[:, :K]), O.MODE_INT4)
     _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, (N,))
     assert_bf16_close(bits(y), y_o)
+
+
+# ------------------------------------------------------ 3-bit KV attention
+def _attn_case(rng, Bq, H, D, T, keep):
+    k_bits = W.normal_bf16(rng, (T, H, D))
+    v_bits = W.normal_bf16(rng, (T, H, D))
+    q = W.normal_bf16(rng, (Bq, H, D))
+    ks, vs = O.kv_quant_3bit(k_bits, keep), O.kv_quant_3bit(v_bits, keep)
+    return q, ks, vs
+
+
+def _check_attention(q, ks, vs, keep):
+    D = q.shape[2]
+    dev = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(DEV)
+    kd = (dev(ks[0]), dev(ks[1]) if len(keep) else None, dev(ks[2]))
+    vd = (dev(vs[0]), dev(vs[1]) if len(keep) else None, dev(vs[2]))
+    kp = torch.tensor(keep, dtype=torch.int32, device=DEV) if len(keep) else None
+    out = B.kv_attention_3bit(dev_bf16(q), kd, vd, kp)
+    torch.cuda.synchronize()
+    want = O.kv_attention_f64(q, ks, vs, keep)
+    got = O.bf16_to_f32(bits(out)).astype(np.float64)
+    vmax = np.abs(O.kv_dequant(*vs, keep, D)).max()
+    # one bf16 ulp of the exact value, plus the fp32 accumulation bound
+    ulp = np.spacing(np.abs(O.bf16_to_f32(O.f64_to_bf16(want))).astype(np.float32)).astype(np.float64) * 2 ** 16
+    err = np.abs(got - want)
+    assert np.all(err <= ulp + 2.5e-4 * vmax), f"max excess {np.max(err - ulp - 2.5e-4 * vmax)}"
+
+
+@pytest.mark.parametrize("Bq,H,D,T,keep", [
+    (1, 1, 128, 1, (0,)), (1, 2, 64, 37, ()), (3, 4, 128, 300, (0, 5, 130)), (8, 2, 256, 513, (0,)),
+    (11, 3, 128, 1000, (0, 999)), (1, 4, 128, 4096, (0,)), (2, 1, 64, 129, tuple(range(0, 129, 3)))])
+def test_kv_attention_parity(Bq, H, D, T, keep):
+    q, ks, vs = _attn_case(np.random.default_rng(Bq * 100 + T), Bq, H, D, T, keep)
+    _check_attention(q, ks, vs, keep)
+
+
+@pytest.mark.parametrize("Bq", [1, 8])
+def test_kv_attention_full_size(Bq):
+    """The decode layer's cache: 4096 tokens x 32 heads x 128, bos at 4 bits,
+    K and V quantised by the library's own kernel."""
+    d = W.decode_layer(batch=1, make_weights=False)
+    keep = torch.tensor([0], dtype=torch.int32, device=DEV)
+    kst = B.kv_quant_3bit(dev_bf16(d["k_cache"]), keep)
+    vst = B.kv_quant_3bit(dev_bf16(d["v_cache"]), keep)
+    q = W.normal_bf16(np.random.default_rng(9), (Bq, 32, 128))
+    out = B.kv_attention_3bit(dev_bf16(q), kst, vst, keep)
+    torch.cuda.synchronize()
+    ks = tuple(host(t) for t in kst)
+    vs = tuple(host(t) for t in vst)
+    want = O.kv_attention_f64(q, ks, vs, (0,))
+    got = O.bf16_to_f32(bits(out)).astype(np.float64)
+    vmax = np.abs(O.kv_dequant(*vs, (0,), 128)).max()
+    ulp = np.spacing(np.abs(O.bf16_to_f32(O.f64_to_bf16(want))).astype(np.float32)).astype(np.float64) * 2 ** 16
+    assert np.all(np.abs(got - want) <= ulp + 2.5e-4 * vmax)
