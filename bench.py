@@ -73,7 +73,7 @@ def parse():
                     help="launch without programmatic dependent launch (each kernel waits for "
                          "the previous one before it starts)")
     ap.add_argument("--section", default=None,
-                    help="run only one breakdown section (o_proj, down_proj, decode, kv), e.g. "
+                    help="run only one breakdown section (o_proj, down_proj, decode, kv, kv_attn), e.g. "
                          "to profile its kernels; prints that section's JSON")
     return ap.parse_args()
 
@@ -517,7 +517,7 @@ def _dev_bf16(torch, bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
 
-SECTIONS = ("o_proj", "down_proj", "decode", "kv")
+SECTIONS = ("o_proj", "down_proj", "decode", "kv", "kv_attn")
 
 
 def breakdown(ctx, args, sections=SECTIONS):
@@ -742,6 +742,32 @@ def section_kv(B, torch, dev, stream, peaks, steps, warm):
                                          "GBps": round(kb / k["kv"] / 1e6, 1),
                                          "frac_hbm": round(kb / k["kv"] / 1e6 / hbm, 4)}
     return out
+
+
+def section_kv_attn(B, torch, dev, stream, peaks, steps, warm):
+    """Decode attention over the 3-bit cache of one layer (K and V [4096 x 32
+    x 128], bos at 4 bits) for 1 and 8 queries per head."""
+    import workloads as W
+    hbm = peaks["hbm_gbs"]
+    kvd = W.decode_layer(batch=1, make_weights=False)
+    T, H, Dh = kvd["k_cache"].shape
+    keep = torch.tensor([0], dtype=torch.int32, device=dev)
+    k_src, v_src = _dev_bf16(torch, kvd["k_cache"], dev), _dev_bf16(torch, kvd["v_cache"], dev)
+    R = 12  # cache replicas: 12 x 13.6 MB > L2
+    stores = [(B.kv_quant_3bit(k_src, keep), B.kv_quant_3bit(v_src, keep)) for _ in range(R)]
+    del k_src, v_src
+    cache_bytes = 2 * (T * H * 3 * Dh // 8 + T * H * 4 + H * Dh // 2)
+    out = {}
+    for nq in (1, 8):
+        q = _dev_bf16(torch, W.normal_bf16(np.random.default_rng(nq), (nq, H, Dh)), dev)
+        o = torch.empty((nq, H, Dh), dtype=torch.bfloat16, device=dev)
+        ms = time_calls(torch, stream, [(lambda r=r: B.kv_attention_3bit(q, stores[r][0], stores[r][1], keep,
+                                                                             out=o)) for r in range(R)],
+                        steps, warm)
+        byt = cache_bytes + 2 * 2 * nq * H * Dh
+        out[f"queries{nq}"] = {"us": round(ms * 1e3, 2), "GBps": round(byt / ms / 1e6, 1),
+                               "frac_hbm": round(byt / ms / 1e6 / hbm, 4)}
+    return {"kv_attention_3bit_4096x32x128": dict(cache_bytes=cache_bytes, **out)}
 
 
 def main():

@@ -48,7 +48,8 @@ _SIGS = {
     "bitlinear_gemm_w2a8_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
     "bitlinear_gemm_w2fp4_acc": ([_P, _P, _I64, _I64, _I64, _P, _P, _P], _INT),
     "bitlinear_gemv_w2": ([_P, _P, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P], _INT),
-    "kv_attention_3bit": ([_P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P], _INT),
+    "kv_attention_3bit": ([_P, _I64, _I64, _I64, _I64, _P, _P, _P, _P, _P, _P, _P, _I64, _P, _P, _P],
+                          _INT),
     "bitlinear_gemv_w2_quant": ([_P, _P, _I64, _INT, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P],
                                 _INT),
     "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
@@ -281,7 +282,7 @@ def kv_quant_3bit(kv: torch.Tensor, keep4_pos: torch.Tensor | None, codes3=None,
 
 
 def kv_attention_3bit(q: torch.Tensor, k_store, v_store, keep4_pos: torch.Tensor | None, out=None,
-                      stream=None):
+                      status=None, stream=None):
     """Decode attention of q [B x H x D] (bf16) over a 3-bit KV cache; k_store
     and v_store are the (codes3, codes4, scale) triples of kv_quant_3bit."""
     k3, k4, ks = k_store
@@ -294,8 +295,10 @@ def kv_attention_3bit(q: torch.Tensor, k_store, v_store, keep4_pos: torch.Tensor
     n4 = 0 if keep4_pos is None else keep4_pos.numel()
     if out is None:
         out = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
+    if status is None:
+        status = status_buffer(q.device)
     _check(lib().kv_attention_3bit(_ptr(q), B, H, D, T, _ptr(k3), _ptr(k4), _ptr(ks), _ptr(v3), _ptr(v4),
-                                   _ptr(vs), _ptr(keep4_pos), n4, _ptr(out), _stream(stream)))
+                                   _ptr(vs), _ptr(keep4_pos), n4, _ptr(out), _ptr(status), _stream(stream)))
     return out
 
 

@@ -346,10 +346,11 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
 int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
                       const uint8_t* k_codes3, const uint8_t* k_codes4, const float* k_scale,
                       const uint8_t* v_codes3, const uint8_t* v_codes4, const float* v_scale,
-                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out,
+                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out, int* dev_status,
                       bitlinear_stream_t stream) {
   if (B < 0 || H <= 0 || T <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: bad sizes");
-  if (D != 64 && D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: D must be 64, 128 or 256");
+  if (D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: D must be 128 or 256");
+  if (H % 4 != 0) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: H must be a multiple of 4");
   if (n_keep4 < 0 || n_keep4 > T || (n_keep4 > 0 && (!keep4_pos || !k_codes4 || !v_codes4)))
     return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: bad 4-bit token list");
   if (n_keep4 > 1024) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_attention_3bit: at most 1024 tokens at 4 bits");
@@ -358,11 +359,14 @@ int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_
   if (B == 0) return ok();
   if (!q || !k_codes3 || !k_scale || !v_codes3 || !v_scale || !out)
     return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: null pointer");
-  if (!aligned16(q) || !aligned16(k_codes3) || !aligned16(v_codes3) || !aligned16(out))
-    return fail(BITLINEAR_ERR_ALIGNMENT, "kv_attention_3bit: q, codes and out must be 16-byte aligned");
+  if (!aligned16(q) || !aligned16(k_codes3) || !aligned16(v_codes3) || !aligned16(k_scale) ||
+      !aligned16(v_scale) || !aligned16(out))
+    return fail(BITLINEAR_ERR_ALIGNMENT, "kv_attention_3bit: q, codes, scales and out must be 16-byte aligned");
+  const char* why = nullptr;
   cudaError_t e = blt::launch_kv_attention(q, B, H, D, T, k_codes3, k_codes4, k_scale, v_codes3,
-                                           v_codes4, v_scale, keep4_pos, n_keep4, out, stream);
-  return e == cudaSuccess ? ok() : cuda_fail(e, "kv_attention_3bit launch");
+                                           v_codes4, v_scale, keep4_pos, n_keep4, out, dev_status,
+                                           static_cast<uint64_t>(g_timeout_ns), stream, &why);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "kv_attention_3bit", why);
 }
 
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream) {

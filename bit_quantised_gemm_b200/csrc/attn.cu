@@ -8,17 +8,22 @@
 //
 // Work split ("split-T"): a cluster of S CTAs owns one head and one group of
 // up to BG queries; CTA r of the cluster walks tokens [T r / S, T (r+1) / S)
-// in tiles of 128 with an online softmax (running max m, running sum l and
+// in tiles of 256 with an online softmax (running max m, running sum l and
 // the running weighted value sum o per query), and the S partial results are
 // merged through distributed shared memory by cluster rank 0, so no global
-// scratch is needed. Within a tile:
-//   * thread i owns token i: it loads the token's packed K row (3D/8 bytes,
-//     8-byte loads) and its scale, and forms s_b for every query b against
-//     the queries held in shared memory (broadcast reads); the codes become
-//     floats with one OR and one subtract (2^23 + code trick);
+// scratch is needed.
+//
+// The rows of one head are 3D/8 bytes every H * 3D/8 bytes in the cache, so
+// each tile's K rows, V rows and their scales arrive by TMA (2-D boxes of 256
+// rows) into a two-stage ring: the next tile is in flight while the current
+// one is computed. Within a tile:
+//   * thread i owns token i: it reads the token's packed K row from shared
+//     memory and forms s_b for every query b against the queries held in
+//     shared memory (broadcast reads); codes become floats with one OR and
+//     one subtract (2^23 + code trick);
 //   * the block reduces the tile maximum and the sum of exp per query;
-//   * the V rows of the tile are staged in shared memory; thread d then
-//     accumulates dimension d over the tile's tokens.
+//   * thread (half, d) accumulates dimension d over half of the tile's
+//     tokens straight from the staged V rows; the halves meet in shared memory.
 #include <cmath>
 
 #include "common.cuh"
@@ -28,19 +33,43 @@
 namespace blt {
 namespace attn {
 
-constexpr int TT = 128;             // tokens per tile = threads per CTA
+constexpr int TT = 256;             // tokens per tile = threads per CTA
+constexpr int VT = 128;             // threads per half in the value pass
+constexpr int NS = 2;               // tile stages
 constexpr int MAX_BG = 8;           // queries per CTA
 constexpr int MAX_KEEP = 1024;      // 4-bit token list held in shared memory
 
 struct Params {
   const uint16_t* q;                // bf16 [B x H x D]
-  const uint8_t* k3; const uint8_t* k4; const float* ks;
-  const uint8_t* v3; const uint8_t* v4; const float* vs;
+  const uint8_t* k4; const uint8_t* v4;  // 4-bit rows [n4 x H x D/2]
   const int32_t* keep4;
   int n4;
   int B, H, T;
   float qk_scale;                   // 1 / sqrt(D)
   uint16_t* out;                    // bf16 [B x H x D]
+  int* status;
+  uint64_t timeout_ns;
+};
+
+template <int D, int BG>
+struct Smem {
+  static constexpr int RB = 3 * D / 8;   // packed 3-bit row bytes
+  uint8_t krow[NS][TT][RB];         // staged K rows of the tile (TMA)
+  uint8_t vrow[NS][TT][RB];         // staged V rows
+  float ksc[NS][TT][4];             // scales of the 4-head group holding h
+  float vsc[NS][TT][4];
+  float qs[BG][D];                  // queries, pre-scaled by 1/sqrt(D)
+  float pv[BG][TT];                 // softmax weight x value scale of the tile's tokens
+  int k4_tok[TT];                   // the tile's 4-bit tokens: list index ...
+  float k4_w[BG][TT];               // ... and softmax weight x value scale
+  float red[TT / 32][BG];
+  float stat[2][BG];                // tile max / sum broadcast
+  int32_t s_keep[MAX_KEEP];
+  float part_m[BG], part_l[BG];
+  float part_o[BG][D];
+  float vpart[BG][D];               // second half of the value pass
+  uint64_t full[NS];
+  int k4_n;
 };
 
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
@@ -78,33 +107,48 @@ __device__ __forceinline__ int keep_index(const int32_t* list, int n, int t) {
 
 template <int D, int BG>
 __global__ void __launch_bounds__(TT)
-kv_attention_kernel(const Params p) {
-  constexpr int RB = 3 * D / 8;     // packed 3-bit row bytes
-  constexpr int NW = RB / 4;        // ... in 32-bit words
-  constexpr int DPT = D / TT > 0 ? D / TT : 1;  // value dims per thread (D = 256: 2)
-  __shared__ float qs[BG][D];       // queries, pre-scaled by 1/sqrt(D)
-  __shared__ float pv[BG][TT];      // softmax weight x value scale of the tile's tokens
-  __shared__ __align__(16) uint32_t vrow[TT][NW + 1];  // the tile's packed V rows (padded)
-  __shared__ int vkeep[TT];         // 4-bit list index of the tile's tokens, or -1
-  __shared__ float red[TT / 32][BG];
-  __shared__ float stat[2][BG];     // tile max / sum broadcast
-  __shared__ int32_t s_keep[MAX_KEEP];
-  __shared__ float part_m[BG], part_l[BG];
-  __shared__ float part_o[BG][D];
+kv_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmKs, const __grid_constant__ CUtensorMap tmVs,
+                    const Params p) {
+  using SM = Smem<D, BG>;
+  constexpr int RB = SM::RB;
+  constexpr int NW = RB / 4;        // packed row in 32-bit words
+  constexpr int DPT = D / VT;       // value dims per thread
+  constexpr uint32_t STAGE_TX = 2 * TT * RB + 2 * TT * 16;
+  extern __shared__ __align__(128) uint8_t smem_raw[];
+  SM& sm = *reinterpret_cast<SM*>(smem_raw);
 
-  pdl_wait();  // the queries and the cache come from earlier kernels
-  pdl_trigger();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_ctarank();
   const int S = static_cast<int>(gridDim.x);
   const int h = blockIdx.y;
+  const int h4 = h & ~3, hl = h & 3;
   const int b0 = blockIdx.z * BG;
   const int nb = min(BG, p.B - b0);
   const int t_begin = static_cast<int>((static_cast<int64_t>(p.T) * rank) / S);
   const int t_end = static_cast<int>((static_cast<int64_t>(p.T) * (rank + 1)) / S);
+  const int n_tiles = (t_end - t_begin + TT - 1) / TT;
   const int n4 = min(p.n4, MAX_KEEP);
 
-  for (int i = tid; i < n4; i += TT) s_keep[i] = __ldg(p.keep4 + i);
+  if (tid == 0) {
+    for (int i = 0; i < NS; ++i) mbar_init(&sm.full[i], 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();  // the queries and the cache come from earlier kernels
+  pdl_trigger();
+  auto issue = [&](int k) {  // thread 0: tile k into stage k % NS
+    const int st = k % NS, t0 = t_begin + k * TT;
+    mbar_arrive_expect_tx(&sm.full[st], STAGE_TX);
+    tma_load_2d(&sm.krow[st][0][0], &tmK, &sm.full[st], h * RB, t0);
+    tma_load_2d(&sm.vrow[st][0][0], &tmV, &sm.full[st], h * RB, t0);
+    tma_load_2d(&sm.ksc[st][0][0], &tmKs, &sm.full[st], h4, t0);
+    tma_load_2d(&sm.vsc[st][0][0], &tmVs, &sm.full[st], h4, t0);
+  };
+  if (tid == 0)
+    for (int k = 0; k < min(NS, n_tiles); ++k) issue(k);
+
+  for (int i = tid; i < n4; i += TT) sm.s_keep[i] = __ldg(p.keep4 + i);
   for (int i = tid; i < BG * D; i += TT) {
     const int b = i / D, d = i - b * D;
     float v = 0.f;
@@ -112,7 +156,7 @@ kv_attention_kernel(const Params p) {
       const uint16_t bits = __ldg(p.q + (static_cast<int64_t>(b0 + b) * p.H + h) * D + d);
       v = __fmul_rn(__uint_as_float(static_cast<uint32_t>(bits) << 16), p.qk_scale);
     }
-    qs[b][d] = v;
+    sm.qs[b][d] = v;
   }
   __syncthreads();
 
@@ -125,27 +169,30 @@ kv_attention_kernel(const Params p) {
     for (int j = 0; j < DPT; ++j) o_run[b][j] = 0.f;
   }
 
-  for (int t0 = t_begin; t0 < t_end; t0 += TT) {
+  bool ok = true;
+  int k = 0;
+  for (; k < n_tiles; ++k) {
+    const int st = k % NS, t0 = t_begin + k * TT;
+    if (!mbar_wait(&sm.full[st], (k / NS) & 1, p.timeout_ns, nullptr)) ok = false;
+    if (__syncthreads_or(!ok)) { ok = false; break; }  // the whole block leaves together
     // ---- scores: thread tid owns token t
     const int t = t0 + tid;
     const bool valid = t < t_end;
+    const int kj = (valid && n4 > 0) ? keep_index(sm.s_keep, n4, t) : -1;
+    const float vsc = sm.vsc[st][tid][hl];
     float s[BG];
-    int kj = -1;
-    float vsc = 0.f;
     if (valid) {
-      const int64_t row = static_cast<int64_t>(t) * p.H + h;
-      kj = n4 > 0 ? keep_index(s_keep, n4, t) : -1;
-      const float ksc = __ldg(p.ks + row);
-      vsc = __ldg(p.vs + row);
-      float acc[BG];
+      float acc[BG][4];  // four independent chains per query
 #pragma unroll
-      for (int b = 0; b < BG; ++b) acc[b] = 0.f;
+      for (int b = 0; b < BG; ++b)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[b][u] = 0.f;
       if (kj < 0) {
         uint32_t w[NW + 1];
-        const uint2* src = reinterpret_cast<const uint2*>(p.k3 + row * RB);
+        const uint2* src = reinterpret_cast<const uint2*>(&sm.krow[st][tid][0]);
 #pragma unroll
         for (int i = 0; i < NW / 2; ++i) {
-          const uint2 u = __ldg(src + i);
+          const uint2 u = src[i];
           w[2 * i] = u.x;
           w[2 * i + 1] = u.y;
         }
@@ -154,32 +201,25 @@ kv_attention_kernel(const Params p) {
         for (int d = 0; d < D; ++d) {
           const float c = code3f(w, d);
 #pragma unroll
-          for (int b = 0; b < BG; ++b) acc[b] = fmaf(qs[b][d], c, acc[b]);
+          for (int b = 0; b < BG; ++b) acc[b][d & 3] = fmaf(sm.qs[b][d], c, acc[b][d & 3]);
         }
-        // the V row of this token, for the value pass
-        const uint2* vsrc = reinterpret_cast<const uint2*>(p.v3 + row * RB);
-#pragma unroll
-        for (int i = 0; i < NW / 2; ++i) {
-          const uint2 u = __ldg(vsrc + i);
-          vrow[tid][2 * i] = u.x;
-          vrow[tid][2 * i + 1] = u.y;
-        }
-        vrow[tid][NW] = 0u;
       } else {
         const uint8_t* k4row = p.k4 + (static_cast<int64_t>(kj) * p.H + h) * (D / 2);
         for (int d = 0; d < D; ++d) {
           const float c = code4f(k4row, d);
 #pragma unroll
-          for (int b = 0; b < BG; ++b) acc[b] = fmaf(qs[b][d], c, acc[b]);
+          for (int b = 0; b < BG; ++b) acc[b][d & 3] = fmaf(sm.qs[b][d], c, acc[b][d & 3]);
         }
       }
+      const float ksc = sm.ksc[st][tid][hl];
 #pragma unroll
-      for (int b = 0; b < BG; ++b) s[b] = __fmul_rn(acc[b], ksc);
+      for (int b = 0; b < BG; ++b)
+        s[b] = __fmul_rn((acc[b][0] + acc[b][1]) + (acc[b][2] + acc[b][3]), ksc);
     } else {
 #pragma unroll
       for (int b = 0; b < BG; ++b) s[b] = -INFINITY;
     }
-    vkeep[tid] = valid ? kj : -2;  // -2: no token
+    if (tid == 0) sm.k4_n = 0;
 
     // ---- tile maximum per query
 #pragma unroll
@@ -187,94 +227,135 @@ kv_attention_kernel(const Params p) {
       float v = s[b];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xFFFFFFFFu, v, o));
-      if (lane == 0) red[warp][b] = v;
+      if (lane == 0) sm.red[warp][b] = v;
     }
     __syncthreads();
     if (tid < BG) {
-      float v = red[0][tid];
+      float v = sm.red[0][tid];
 #pragma unroll
-      for (int w = 1; w < TT / 32; ++w) v = fmaxf(v, red[w][tid]);
-      stat[0][tid] = v;
+      for (int w = 1; w < TT / 32; ++w) v = fmaxf(v, sm.red[w][tid]);
+      sm.stat[0][tid] = v;
     }
     __syncthreads();
     float m_new[BG], corr[BG];
 #pragma unroll
     for (int b = 0; b < BG; ++b) {
-      m_new[b] = fmaxf(m_run[b], stat[0][b]);
+      m_new[b] = fmaxf(m_run[b], sm.stat[0][b]);
       corr[b] = expf(m_run[b] - m_new[b]);  // 0 on the first tile (m_run = -inf)
       const float e = valid ? expf(s[b] - m_new[b]) : 0.f;
-      pv[b][tid] = __fmul_rn(e, vsc);
+      // absent and 4-bit tokens weigh nothing in the 3-bit value pass
+      sm.pv[b][tid] = kj < 0 ? __fmul_rn(e, vsc) : 0.f;
+      s[b] = __fmul_rn(e, vsc);  // kept for a 4-bit token below
       float v = e;
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
-      if (lane == 0) red[warp][b] = v;
+      if (lane == 0) sm.red[warp][b] = v;
     }
     __syncthreads();
     if (tid < BG) {
-      float v = red[0][tid];
+      float v = sm.red[0][tid];
 #pragma unroll
-      for (int w = 1; w < TT / 32; ++w) v += red[w][tid];
-      stat[1][tid] = v;
+      for (int w = 1; w < TT / 32; ++w) v += sm.red[w][tid];
+      sm.stat[1][tid] = v;
+    }
+    if (kj >= 0) {  // a 4-bit token of this tile (rare): its own list for the value pass
+      const int slot = atomicAdd(&sm.k4_n, 1);
+      sm.k4_tok[slot] = kj;
+#pragma unroll
+      for (int b = 0; b < BG; ++b) sm.k4_w[b][slot] = s[b];
     }
     __syncthreads();
 #pragma unroll
     for (int b = 0; b < BG; ++b) {
-      l_run[b] = fmaf(l_run[b], corr[b], stat[1][b]);
+      l_run[b] = fmaf(l_run[b], corr[b], sm.stat[1][b]);
       m_run[b] = m_new[b];
     }
 
-    // ---- values: thread tid owns dimensions d = tid + TT j
-    const int ntok = min(TT, t_end - t0);
+    // ---- values: thread tid owns dimensions d = dl + VT j of one half of the
+    // tile's tokens (half = tid / VT), read straight from the staged rows
+    // (rows with weight 0 add nothing), with four independent chains.
+    const int nk4 = sm.k4_n;
+    const int half = tid / VT, dl = tid % VT;
+    float vsum[BG][DPT];
 #pragma unroll
     for (int j = 0; j < DPT; ++j) {
-      const int d = tid + TT * j;
-      if (d >= D) break;
-      float acc[BG];
+      const int d = dl + VT * j;
+      float acc[BG][4];
 #pragma unroll
-      for (int b = 0; b < BG; ++b) acc[b] = 0.f;
+      for (int b = 0; b < BG; ++b)
+#pragma unroll
+        for (int u = 0; u < 4; ++u) acc[b][u] = 0.f;
       const int bit = 3 * d, wi = bit >> 5, sh = bit & 31;
-      for (int i = 0; i < ntok; ++i) {
-        float c;
-        const int kk = vkeep[i];
-        if (kk < 0) {
-          uint32_t v = vrow[i][wi] >> sh;
-          if (sh > 29) v |= vrow[i][wi + 1] << (32 - sh);
-          c = __int_as_float(static_cast<int>((v & 7u) | 0x4B000000u)) - 8388612.f;
-        } else {
-          c = code4f(p.v4 + (static_cast<int64_t>(kk) * p.H + h) * (D / 2), d);
-        }
+      const int i0 = half * VT;
+      const uint8_t* vbase = &sm.vrow[st][0][0];
+#pragma unroll 4
+      for (int i = i0; i < i0 + VT; i += 4) {
 #pragma unroll
-        for (int b = 0; b < BG; ++b) acc[b] = fmaf(pv[b][i], c, acc[b]);
+        for (int u = 0; u < 4; ++u) {
+          const uint32_t* row = reinterpret_cast<const uint32_t*>(vbase + (i + u) * RB);
+          uint32_t v = row[wi] >> sh;
+          if (sh > 29) v |= row[wi + 1] << (32 - sh);
+          const float c = __int_as_float(static_cast<int>((v & 7u) | 0x4B000000u)) - 8388612.f;
+#pragma unroll
+          for (int b = 0; b < BG; ++b) acc[b][u] = fmaf(sm.pv[b][i + u], c, acc[b][u]);
+        }
+      }
+      for (int kk = half; kk < nk4; kk += 2) {
+        const float c = code4f(p.v4 + (static_cast<int64_t>(sm.k4_tok[kk]) * p.H + h) * (D / 2), d);
+#pragma unroll
+        for (int b = 0; b < BG; ++b) acc[b][0] = fmaf(sm.k4_w[b][kk], c, acc[b][0]);
       }
 #pragma unroll
-      for (int b = 0; b < BG; ++b) o_run[b][j] = fmaf(o_run[b][j], corr[b], acc[b]);
+      for (int b = 0; b < BG; ++b) vsum[b][j] = (acc[b][0] + acc[b][1]) + (acc[b][2] + acc[b][3]);
     }
-    __syncthreads();  // the tile's shared rows are reused by the next tile
+    if (half == 1) {
+#pragma unroll
+      for (int j = 0; j < DPT; ++j)
+#pragma unroll
+        for (int b = 0; b < BG; ++b) sm.vpart[b][dl + VT * j] = vsum[b][j];
+    }
+    __syncthreads();  // every thread is done with stage st; the halves meet
+    if (half == 0) {
+#pragma unroll
+      for (int j = 0; j < DPT; ++j)
+#pragma unroll
+        for (int b = 0; b < BG; ++b)
+          o_run[b][j] = fmaf(o_run[b][j], corr[b], vsum[b][j] + sm.vpart[b][dl + VT * j]);
+    }
+    if (tid == 0 && k + NS < n_tiles) issue(k + NS);  // refill the stage just read
+  }
+  if (!ok) {
+    report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
+    // copies still in flight land before the block's shared memory is released
+    if (tid == 0)
+      for (int j = k; j < min(k + NS, n_tiles); ++j)
+        mbar_wait(&sm.full[j % NS], (j / NS) & 1, p.timeout_ns, nullptr);
   }
 
   // ---- merge the S partial results on cluster rank 0
   // every thread holds the same m_run / l_run; thread b publishes query b
 #pragma unroll
   for (int b = 0; b < BG; ++b)
-    if (tid == b) { part_m[b] = m_run[b]; part_l[b] = l_run[b]; }
+    if (tid == b) { sm.part_m[b] = m_run[b]; sm.part_l[b] = l_run[b]; }
+  if (tid < VT) {  // the value sums live in the first half
 #pragma unroll
-  for (int b = 0; b < BG; ++b)
+    for (int b = 0; b < BG; ++b)
 #pragma unroll
-    for (int j = 0; j < DPT; ++j)
-      if (tid + TT * j < D) part_o[b][tid + TT * j] = o_run[b][j];
+      for (int j = 0; j < DPT; ++j) sm.part_o[b][tid + VT * j] = o_run[b][j];
+  }
   cluster_sync();
-  if (rank == 0) {
+  if (rank == 0 && ok) {
     for (int i = tid; i < nb * D; i += TT) {
       const int b = i / D, d = i - b * D;
       float M = -INFINITY;
       for (int r = 0; r < S; ++r)
-        M = fmaxf(M, ld_dsmem_f32(map_shared_rank(smem_u32(&part_m[b]), r)));
+        M = fmaxf(M, ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_m[b]), r)));
       float num = 0.f, den = 0.f;
       for (int r = 0; r < S; ++r) {
-        const float mr = ld_dsmem_f32(map_shared_rank(smem_u32(&part_m[b]), r));
+        const float mr = ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_m[b]), r));
         const float w = mr == -INFINITY ? 0.f : expf(mr - M);
-        den = fmaf(w, ld_dsmem_f32(map_shared_rank(smem_u32(&part_l[b]), r)), den);
-        num = fmaf(w, ld_dsmem_f32(map_shared_rank(smem_u32(&part_o[b][d]), r)), num);
+        den = fmaf(w, ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_l[b]), r)), den);
+        num = fmaf(w, ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_o[b][d]), r)), num);
       }
       p.out[(static_cast<int64_t>(b0 + b) * p.H + h) * D + d] =
           __bfloat16_as_ushort(__float2bfloat16_rn(num / den));
@@ -286,21 +367,62 @@ kv_attention_kernel(const Params p) {
 }  // namespace attn
 
 template <int D, int BG>
-static cudaError_t launch_attn_t(const attn::Params& p, int S, cudaStream_t s) {
+static cudaError_t launch_attn_t(const CUtensorMap (&maps)[4], const attn::Params& p, int S,
+                                 cudaStream_t s) {
+  static bool attr_set = false;  // once per process (not during graph capture)
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(attn::kv_attention_kernel<D, BG>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(sizeof(attn::Smem<D, BG>)));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
   const dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(p.H),
                   static_cast<unsigned>((p.B + BG - 1) / BG));
-  return launch_kernel(attn::kv_attention_kernel<D, BG>, grid, dim3(attn::TT), 0, s,
-                       static_cast<unsigned>(S), p);
+  return launch_kernel(attn::kv_attention_kernel<D, BG>, grid, dim3(attn::TT),
+                       sizeof(attn::Smem<D, BG>), s, static_cast<unsigned>(S), maps[0], maps[1],
+                       maps[2], maps[3], p);
 }
 
 cudaError_t launch_kv_attention(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
                                 const uint8_t* k3, const uint8_t* k4, const float* ks,
                                 const uint8_t* v3, const uint8_t* v4, const float* vs,
-                                const int32_t* keep4, int64_t n4, uint16_t* out, cudaStream_t s) {
+                                const int32_t* keep4, int64_t n4, uint16_t* out, int* status,
+                                uint64_t timeout_ns, cudaStream_t s, const char** why) {
+  EncodeTiledFn enc = get_encode_tiled();
+  if (!enc) { *why = "cuTensorMapEncodeTiled unavailable"; return cudaErrorNotSupported; }
+  const uint64_t RB = static_cast<uint64_t>(3 * D / 8);
+  CUtensorMap maps[4];
+  // packed rows: [T rows][H * RB bytes]; a box = 256 rows x RB bytes (one head)
+  for (int i = 0; i < 2; ++i) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H) * RB, static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * RB};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(RB), static_cast<cuuint32_t>(attn::TT)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(i == 0 ? k3 : v3), dims,
+            strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled rejected the packed cache layout";
+      return cudaErrorInvalidValue;
+    }
+  }
+  // scales: [T rows][H floats]; a box = 256 rows x the 4 heads holding h
+  for (int i = 0; i < 2; ++i) {
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(T)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(H) * 4};
+    const cuuint32_t box[2] = {4, static_cast<cuuint32_t>(attn::TT)};
+    const cuuint32_t estr[2] = {1, 1};
+    if (enc(&maps[2 + i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(i == 0 ? ks : vs),
+            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS) {
+      *why = "cuTensorMapEncodeTiled rejected the scale layout";
+      return cudaErrorInvalidValue;
+    }
+  }
   attn::Params p{};
   p.q = q;
-  p.k3 = k3; p.k4 = k4; p.ks = ks;
-  p.v3 = v3; p.v4 = v4; p.vs = vs;
+  p.k4 = k4;
+  p.v4 = v4;
   p.keep4 = keep4;
   p.n4 = static_cast<int>(n4);
   p.B = static_cast<int>(B);
@@ -308,14 +430,16 @@ cudaError_t launch_kv_attention(const uint16_t* q, int64_t B, int64_t H, int64_t
   p.T = static_cast<int>(T);
   p.qk_scale = static_cast<float>(1.0 / std::sqrt(static_cast<double>(D)));
   p.out = out;
+  p.status = status;
+  p.timeout_ns = timeout_ns;
   const int BG = B == 1 ? 1 : attn::MAX_BG;
   const int64_t ctas = H * ((B + BG - 1) / BG);
-  // split T over a cluster until the grid fills the SMs (and each CTA keeps a full tile)
+  // split T over a cluster while the grid stays within two waves and every
+  // CTA keeps at least one full tile
   int S = 1;
   while (S < 8 && ctas * S * 2 <= 2 * num_sms() && T / (2 * S) >= attn::TT) S *= 2;
-  if (D == 64) return BG == 1 ? launch_attn_t<64, 1>(p, S, s) : launch_attn_t<64, 8>(p, S, s);
-  if (D == 128) return BG == 1 ? launch_attn_t<128, 1>(p, S, s) : launch_attn_t<128, 8>(p, S, s);
-  return BG == 1 ? launch_attn_t<256, 1>(p, S, s) : launch_attn_t<256, 8>(p, S, s);
+  if (D == 128) return BG == 1 ? launch_attn_t<128, 1>(maps, p, S, s) : launch_attn_t<128, 8>(maps, p, S, s);
+  return BG == 1 ? launch_attn_t<256, 1>(maps, p, S, s) : launch_attn_t<256, 8>(maps, p, S, s);
 }
 
 }  // namespace blt

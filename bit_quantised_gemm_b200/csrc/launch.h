@@ -15,7 +15,8 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 cudaError_t launch_kv_attention(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
                                 const uint8_t* k3, const uint8_t* k4, const float* ks,
                                 const uint8_t* v3, const uint8_t* v4, const float* vs,
-                                const int32_t* keep4, int64_t n4, uint16_t* out, cudaStream_t s);
+                                const int32_t* keep4, int64_t n4, uint16_t* out, int* status,
+                                uint64_t timeout_ns, cudaStream_t s, const char** why);
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s);

@@ -213,12 +213,14 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
  *              with the same keep4_pos list (codes4 nullable iff n_keep4 == 0)
  *   keep4_pos  device int32 [n_keep4], strictly increasing, n_keep4 <= 1024
  *   out        device bf16 [B x H x D]
- * Requires D in {64, 128, 256}, T >= 1; B == 0 launches nothing.
+ *   dev_status as for the GEMMs (bounded waits on the cache tiles)
+ * Requires D in {128, 256}, H % 4 == 0, T >= 1, every pointer but codes4 and
+ * keep4_pos 16-byte aligned; B == 0 launches nothing.
  */
 int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
                       const uint8_t* k_codes3, const uint8_t* k_codes4, const float* k_scale,
                       const uint8_t* v_codes3, const uint8_t* v_codes4, const float* v_scale,
-                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out,
+                      const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out, int* dev_status,
                       bitlinear_stream_t stream);
 
 /* Synchronise the stream and read *dev_status: BITLINEAR_OK, or

@@ -114,8 +114,10 @@ def test_kv_attention_argument_errors():
                  keep=None, n4=0, out=FAKE)
         a.update(kw)
         return L.kv_attention_3bit(a["q"], a["B"], a["H"], a["D"], a["T"], a["k3"], a["k4"], a["ks"],
-                                   a["v3"], a["v4"], a["vs"], a["keep"], a["n4"], a["out"], None)
+                                   a["v3"], a["v4"], a["vs"], a["keep"], a["n4"], a["out"], None, None)
     assert call(D=96) == _lib.ERR_UNSUPPORTED
+    assert call(D=64) == _lib.ERR_UNSUPPORTED               # 24-byte rows: no TMA box
+    assert call(H=6) == _lib.ERR_UNSUPPORTED                # scale rows: H % 4
     assert call(T=0) == _lib.ERR_INVALID_ARG
     assert call(n4=1) == _lib.ERR_INVALID_ARG               # no list / 4-bit rows
     assert call(n4=65, keep=FAKE, k4=FAKE, v4=FAKE) == _lib.ERR_INVALID_ARG  # more than T

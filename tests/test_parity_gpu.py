@@ -470,8 +470,9 @@ def _check_attention(q, ks, vs, keep):
 
 
 @pytest.mark.parametrize("Bq,H,D,T,keep", [
-    (1, 1, 128, 1, (0,)), (1, 2, 64, 37, ()), (3, 4, 128, 300, (0, 5, 130)), (8, 2, 256, 513, (0,)),
-    (11, 3, 128, 1000, (0, 999)), (1, 4, 128, 4096, (0,)), (2, 1, 64, 129, tuple(range(0, 129, 3)))])
+    (1, 4, 128, 1, (0,)), (1, 4, 128, 37, ()), (3, 4, 128, 300, (0, 5, 130)), (8, 4, 256, 513, (0,)),
+    (11, 8, 128, 1000, (0, 999)), (1, 4, 128, 4096, (0,)), (2, 4, 128, 129, tuple(range(0, 129, 3))),
+    (1, 4, 256, 2000, ())])
 def test_kv_attention_parity(Bq, H, D, T, keep):
     q, ks, vs = _attn_case(np.random.default_rng(Bq * 100 + T), Bq, H, D, T, keep)
     _check_attention(q, ks, vs, keep)
