@@ -23,12 +23,22 @@
 //
 // Work split. Rows of Wp are contiguous (K/4 bytes each), so an item of RW
 // consecutive output features is one contiguous range, fetched with a single
-// cp.async.bulk into a per-warp ring of SW slots. Items are dealt round-robin
-// over all warps of the grid (neighbouring warps read neighbouring rows). A
-// lane takes the packed words j = lane, lane + 32, ... of every row of the
+// cp.async.bulk into a per-warp ring of `sw` slots. Every CTA owns one
+// contiguous, equal share of the items (the weight bytes per SM are balanced)
+// and deals it round-robin over its warps, so neighbouring warps read
+// neighbouring rows. A lane takes the packed words j = lane, lane + 32, ... of every row of the
 // item, so the 4-byte weight reads of a warp and its 16-byte reads of the
 // activation codes (all MT tokens, held in shared memory for the whole
-// kernel) are contiguous. The RW x MT partial sums of a lane are reduced
+// kernel) are contiguous. With one token and K <= 4096 the activation words
+// a lane needs (the same for every row) are instead loaded straight into its
+// registers after the wait, regrouped there, and their sum is subtracted
+// from the lane's partial sums: no shared-memory copy of the activations, no
+// block-wide barrier, and only 4-byte weight reads in the inner loop. That
+// variant runs as 8-warp CTAs with at most 112 KB of shared memory, two to an
+// SM: the CTA of the next kernel in the stream (launched early through
+// programmatic dependent launch) becomes resident beside this one and has
+// its weights in flight before this kernel ends. The RW x MT partial sums of
+// a lane are reduced
 // across the warp with a transposing butterfly: log2(RW MT) exchange steps
 // that halve the values held per lane, then plain xor steps.
 #include <algorithm>
@@ -40,13 +50,16 @@
 namespace blt {
 namespace gemv_cc {
 
-constexpr int SW = 2;         // ring slots per warp
+constexpr int MAX_SW = 4;             // ring slots per warp, at most
 constexpr int MAX_WARPS = 16;
-constexpr int SMEM_LIMIT = 232448;
+constexpr int SMEM_LIMIT = 232448;   // one CTA per SM
+constexpr int SMEM_PAIR = 114688;    // two CTAs per SM (register-activation variant)
+constexpr int PAIR_WARPS = 8;
 
 struct Params {
   int M, N, K;
   int n_items;
+  int sw;               // ring slots per warp
   const int8_t* xq;     // activation codes [M x K] (codes given)
   const float* xs;
   const uint16_t* x;    // bf16 activations [M x ldx] (quantised here)
@@ -172,9 +185,12 @@ __device__ __forceinline__ float warp_max_f(float v) {
 // FUSED: the kernel quantises the bf16 activations itself (per-token absmax,
 // INT8 / INT4, optionally of the ReLU^2-gated product), redundantly in every
 // CTA, instead of reading codes written by a separate quantiser launch.
-template <int MT, int RW, bool FUSED>
-__global__ void __launch_bounds__(MAX_WARPS * 32, 1)
+// LW > 0: the activation codes are held in registers, LW packed-word
+// columns per lane (K <= 512 LW); codes given (not FUSED) only.
+template <int MT, int RW, bool FUSED, int LW>
+__global__ void __launch_bounds__(LW > 0 ? PAIR_WARPS * 32 : MAX_WARPS * 32, LW > 0 ? 2 : 1)
 bitlinear_gemv_dp4a_kernel(const Params p) {
+  static_assert(LW == 0 || (!FUSED && LW % 4 == 0), "register activations: codes given");
   constexpr int NACC = MT <= 2 ? 4 : 2;
   constexpr int U = MT <= 2 ? 4 : (MT == 4 ? 2 : 1);  // words per lane per batch of loads
   constexpr int NV = RW * MT;
@@ -185,21 +201,23 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
   const int nwarps = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  uint8_t* xsm = smem;                                  // [MT][K] regrouped codes
-  uint8_t* ring = smem + MT * K;                        // [nwarps][SW][slot_bytes]
+  uint8_t* xsm = smem;                                  // [MT][K] regrouped codes (LW == 0)
+  const int SW = p.sw;
+  uint8_t* ring = smem + (LW > 0 ? 0 : MT * K);         // [nwarps][SW][slot_bytes]
   uint64_t* bars = reinterpret_cast<uint64_t*>(ring + nwarps * SW * slot_bytes);
   uint64_t* xbar = bars + nwarps * SW;
   int* xsum = reinterpret_cast<int*>(xbar + 1);         // [MT]
 
   uint8_t* my_ring = ring + warp * SW * slot_bytes;
   uint64_t* my_bar = bars + warp * SW;
-  const int gw = blockIdx.x * nwarps + warp;
-  const int GW = gridDim.x * nwarps;
-  const int n_mine = gw < p.n_items ? (p.n_items - 1 - gw) / GW + 1 : 0;
+  // this CTA's share of the items: [lo, hi)
+  const int lo = static_cast<int>(static_cast<int64_t>(blockIdx.x) * p.n_items / gridDim.x);
+  const int hi = static_cast<int>(static_cast<int64_t>(blockIdx.x + 1) * p.n_items / gridDim.x);
+  const int n_mine = warp < hi - lo ? (hi - lo - 1 - warp) / nwarps + 1 : 0;
+  auto item_of = [&](int s) { return lo + warp + s * nwarps; };
 
   auto issue = [&](int s) {  // lane 0: fetch the s-th item of this warp
-    const int item = gw + s * GW;
-    const int n0 = item * RW;
+    const int n0 = item_of(s) * RW;
     const int rows = min(RW, p.N - n0);
     const uint32_t bytes = static_cast<uint32_t>(rows * row_bytes);
     uint64_t* bar = my_bar + (s % SW);
@@ -216,6 +234,7 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
     fence_mbar_init();
     for (int s = 0; s < min(SW, n_mine); ++s) issue(s);
   }
+  __syncwarp();  // the warp's barriers are initialised before any lane waits on them
   float gam[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) gam[i] = i < p.G ? __ldg(p.gamma + i) : 0.f;
@@ -296,6 +315,10 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
       if (lane == 0 && part[t] != 0) atomicAdd(&xsum[t], part[t]);
     }
     __syncthreads();
+  } else if constexpr (LW > 0) {
+    pdl_wait();  // activation codes and scales come from the previous kernel
+#pragma unroll
+    for (int t = 0; t < MT; ++t) xsc[t] = t < p.M ? __ldg(p.xs + t) : 0.f;
   } else {
     pdl_wait();  // activation codes and scales come from the previous kernel
     if (threadIdx.x == 0) {  // the codes are one contiguous M x K block
@@ -336,12 +359,30 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
     }
     __syncthreads();
   }
+  const int words = K >> 4;
   int xsm_sum[MT];
+  uint4 xr[LW > 0 ? LW : 1][MT];  // LW > 0: this lane's regrouped activation words
+  if constexpr (LW > 0) {
 #pragma unroll
-  for (int t = 0; t < MT; ++t) xsm_sum[t] = xsum[t];
+    for (int t = 0; t < MT; ++t) xsm_sum[t] = 0;
+#pragma unroll
+    for (int i = 0; i < LW; ++i) {
+      const int j = lane + 32 * i;
+#pragma unroll
+      for (int t = 0; t < MT; ++t) {
+        const uint4 v = (j < words && t < p.M)
+                            ? *reinterpret_cast<const uint4*>(p.xq + static_cast<int64_t>(t) * K + 16 * j)
+                            : make_uint4(0u, 0u, 0u, 0u);
+        xsm_sum[t] += byte_sum16(v);  // this lane's share of sum_k x[k]
+        xr[i][t] = regroup16(v);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int t = 0; t < MT; ++t) xsm_sum[t] = xsum[t];
+  }
 
   const uint32_t x_base = smem_u32(xsm);
-  const int words = K >> 4;
   bool timed_out = !x_ok;
   int s = 0;
   for (; s < n_mine && !timed_out; ++s) {
@@ -360,6 +401,22 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 
     // U words per lane are loaded before any arithmetic; words past the row
     // end read as code 0, which adds nothing.
+    if constexpr (LW > 0) {
+#pragma unroll
+      for (int i = 0; i < LW; i += 4) {
+        uint32_t w[4][RW];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int j = lane + 32 * (i + u);
+#pragma unroll
+          for (int r = 0; r < RW; ++r) w[u][r] = j < words ? ld_shared_u32(w_base + r * row_bytes + 4 * j) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+#pragma unroll
+          for (int r = 0; r < RW; ++r) word_dot<MT, NACC>(w[u][r], xr[i + u], acc[r]);
+      }
+    } else
     for (int j0 = lane; j0 < words; j0 += 32 * U) {
       uint4 xv[U][MT];
       uint32_t w[U][RW];
@@ -385,12 +442,13 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 #pragma unroll
     for (int r = 0; r < RW; ++r)
 #pragma unroll
-      for (int t = 0; t < MT; ++t) v[r * MT + t] = combine<NACC>(acc[r][t]);
+      for (int t = 0; t < MT; ++t)
+        v[r * MT + t] = combine<NACC>(acc[r][t]) - (LW > 0 ? xsm_sum[t] : 0);
     int idx;
     const int sum = transpose_reduce<NV>(v, lane, idx);
     if ((lane & (32 / NV - 1)) == 0) {
       const int r = idx / MT, t = idx % MT;
-      const int n = (gw + s * GW) * RW + r;
+      const int n = item_of(s) * RW + r;
       if (t < p.M && n < p.N) {
         int ts = 0;
         float xst = 0.f;
@@ -405,7 +463,7 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
         float gm = gam[0];
 #pragma unroll
         for (int i = 1; i < 8; ++i) gm = (g == i) ? gam[i] : gm;
-        const int acc = sum - ts;
+        const int acc = LW > 0 ? sum : sum - ts;
         p.y[static_cast<int64_t>(t) * p.ldy + n] = __bfloat16_as_ushort(
             __float2bfloat16_rn(static_cast<float>(acc) * (xst * gm)));
       }
@@ -425,47 +483,94 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 
 }  // namespace gemv_cc
 
-static size_t dp4a_smem_bytes(int mt, int rw, int64_t K, int warps) {
-  return size_t(mt) * K + size_t(warps) * gemv_cc::SW * rw * (K / 4) +
-         size_t(warps) * gemv_cc::SW * 8 + 8 + 8 * 4 + size_t(gemv_cc::MAX_WARPS) * mt * 4;
+// xk: bytes of activation codes staged in shared memory (mt K, or 0 when
+// they are held in registers)
+static size_t dp4a_smem_bytes(int mt, int rw, int64_t K, int warps, int sw, int64_t xk) {
+  return size_t(xk) + size_t(warps) * sw * rw * (K / 4) + size_t(warps) * sw * 8 + 8 + 8 * 4 +
+         size_t(gemv_cc::MAX_WARPS) * mt * 4;
 }
 
 static int dp4a_tokens(int64_t M) { return M == 1 ? 1 : M == 2 ? 2 : M <= 4 ? 4 : 8; }
 
-// Largest warp count (<= 16) whose ring fits next to the activation codes;
-// 0 when even one warp does not fit.
-static int dp4a_warps_fit(int mt, int rw, int64_t K) {
-  for (int w = gemv_cc::MAX_WARPS; w >= 1; --w)
-    if (dp4a_smem_bytes(mt, rw, K, w) <= size_t(gemv_cc::SMEM_LIMIT)) return w;
-  return 0;
+struct Dp4aShape {
+  int warps = 0, sw = 0;
+  size_t smem = 0;
+};
+
+// Warps and ring slots for a CTA that owns `per_cta` items: as many warps as
+// there are items (up to the block size), then as many slots as a warp has
+// items (up to 4), inside `limit` bytes of shared memory; fewer slots (not
+// below 2 while a warp has two items or more), then fewer warps, if it does
+// not fit. warps = 0 when even one warp with one slot does not fit.
+static Dp4aShape dp4a_shape(int mt, int rw, int64_t K, int per_cta, int max_warps, size_t limit,
+                            bool x_in_regs = false) {
+  Dp4aShape r;
+  for (int w = std::min(max_warps, std::max(per_cta, 1)); w >= 1; --w) {
+    const int ipw = (per_cta + w - 1) / w;
+    const int top = std::max(1, std::min(gemv_cc::MAX_SW, ipw));
+    const int bottom = std::min(2, top);
+    for (int sw = top; sw >= bottom; --sw) {
+      const size_t b = dp4a_smem_bytes(mt, rw, K, w, sw, x_in_regs ? 0 : mt * K);
+      if (b <= limit) {
+        r.warps = w;
+        r.sw = sw;
+        r.smem = b;
+        return r;
+      }
+    }
+  }
+  return r;
 }
 
 bool gemv_dp4a_supported(int64_t M, int64_t K) {
   if (M < 1 || M > kGemvDp4aMaxTokens || K % 64 != 0) return false;
-  return dp4a_warps_fit(dp4a_tokens(M), 2, K) > 0;
+  return dp4a_shape(dp4a_tokens(M), 2, K, 1, 1, gemv_cc::SMEM_LIMIT).warps > 0;  // staged codes
 }
 
+// One CTA per SM, each with an equal share of the items. One token with
+// K <= 4096 and codes given: activations in registers (8 columns per lane),
+// CTAs sized to share the SM with the next kernel's.
 template <int MT, int RW, bool FUSED>
 static cudaError_t launch_mt(gemv_cc::Params p, cudaStream_t s) {
   p.n_items = (p.N + RW - 1) / RW;
   const int grid = std::min(num_sms(), p.n_items);
-  int warps = (p.n_items + grid - 1) / grid;
-  warps = std::min(warps, dp4a_warps_fit(MT, RW, p.K));
-  const size_t smem = dp4a_smem_bytes(MT, RW, p.K, warps);
-  auto kern = gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED>;
+  const int per_cta = (p.n_items + grid - 1) / grid;
+  constexpr bool kRegs = MT == 1 && !FUSED;
+  const bool regs = kRegs && p.K <= 4096;
+  const Dp4aShape sh =
+      regs ? dp4a_shape(MT, RW, p.K, per_cta, gemv_cc::PAIR_WARPS, gemv_cc::SMEM_PAIR, true)
+           : dp4a_shape(MT, RW, p.K, per_cta, gemv_cc::MAX_WARPS, gemv_cc::SMEM_LIMIT, false);
+  if (sh.warps == 0) return cudaErrorInvalidValue;
+  p.sw = sh.sw;
+  auto kern = regs ? gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED, kRegs ? 8 : 0>
+                   : gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED, 0>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+                                       static_cast<int>(sh.smem));
+  // all of the unified L1 as shared memory, so that a second CTA finds room
+  // without the SM changing its split
+  if (e == cudaSuccess && regs)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return e;
-  return launch_kernel(kern, dim3(grid), dim3(warps * 32), smem, s, 0u, p);
+  return launch_kernel(kern, dim3(grid), dim3(sh.warps * 32), sh.smem, s, 0u, p);
 }
 
-// Items of 4 output features when there are enough of them to give every
-// SM a full complement of warps (and the ring fits), else of 2.
+// Items of 4 output features when every warp of every CTA gets at least one
+// (and two slots per warp fit), else of 2 (more items to spread over the
+// warps).
 template <int MT, bool FUSED>
 static cudaError_t launch_pick_rows(const gemv_cc::Params& p, cudaStream_t s) {
+  if constexpr (MT == 1 && !FUSED) {  // register activations: an item or two per warp
+    if (p.K <= 4096) {
+      if (int64_t(p.N) > int64_t(2) * gemv_cc::PAIR_WARPS * num_sms())
+        return launch_mt<MT, 4, FUSED>(p, s);
+      return launch_mt<MT, 2, FUSED>(p, s);
+    }
+  }
   if constexpr (MT <= 4) {  // eight tokens: 2 rows (registers)
-    if (int64_t(p.N) >= int64_t(4) * gemv_cc::MAX_WARPS * num_sms() &&
-        dp4a_warps_fit(MT, 4, p.K) == gemv_cc::MAX_WARPS)
+    constexpr int W = gemv_cc::MAX_WARPS;
+    if (int64_t(p.N) >= int64_t(4) * W * num_sms() &&
+        dp4a_shape(MT, 4, p.K, 2 * W, W, gemv_cc::SMEM_LIMIT).warps == W)
       return launch_mt<MT, 4, FUSED>(p, s);
   }
   return launch_mt<MT, 2, FUSED>(p, s);
