@@ -11,8 +11,9 @@ value = 2*M*K*N summed over the four GEMMs / step time, in TOPS.
 
 Inputs are already resident in HBM; R replicas of all buffers rotate so the
 working set (>= 270 MB) exceeds the 126 MB L2 between consecutive steps.
-Each replica's step is one CUDA graph. Per-kernel durations come from CUDA
-events captured inside the graphs (last 24 steps of the timed region).
+Each replica's step is one CUDA graph (no event nodes inside). Per-kernel
+durations come from CUDA graphs of 8 back-to-back launches of that kernel
+alone over the replicas, timed the same way.
 
 Also reported (same run, rank 0, unless --no-breakdown): the o_proj top-k
 INT8 GEMM, the down_proj ReLU^2 INT8 GEMM, the decode layer at batch 1/8/64
@@ -358,7 +359,7 @@ def bench_ours(args, ws, rank, local):
         pk = int8_peak if "w2a4" in n else fp4_peak
         kernels[n] = {"us": round(kms[n] * 1e3, 2), "TOPS": round(tops, 1),
                       "frac_of_peak": round(tops / pk, 4),
-                      "peak": "int8" if "w2a4" in n else "fp4 (the f8f6f4 kind runs at the fp8 rate: 0.5 at most)"}
+                      "peak": "int8" if "w2a4" in n else "fp4 (tcgen05 kind::mxf4, block scales 1.0)"}
 
     value = OPS_PER_STEP * args.steps * ws / (ms * 1e-3) / 1e12
     out = {"metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": ws,
@@ -366,7 +367,7 @@ def bench_ours(args, ws, rank, local):
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "s8,e2m1 (x ternary)", "data": "synthetic",
            "config": {"workload": WORKLOAD, "tokens": M_TOK, "d_model": D, "qkv_out": 3 * D,
-                      "gate_up_out": 2 * FFN, "variants": ["INT4 (s8 MMA)", "FP4 e2m1 (f8f6f4 MMA)"],
+                      "gate_up_out": 2 * FFN, "variants": ["INT4 (s8 MMA)", "FP4 e2m1 (mxf4 MMA, unit block scales)"],
                       "parallelism": f"replicas x{ws}",
                       "l2": f"{R} rotating replicas of all inputs/weights/outputs (>270 MB > 126 MB L2)",
                       "graphs": "one CUDA graph per step",

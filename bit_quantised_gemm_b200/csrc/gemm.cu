@@ -1,8 +1,18 @@
 // Prefill BitLinear GEMM on sm_100a tensor cores.
 //
 //   acc[m, n] = sum_k a[m, k] * w[k, n],  a = int8 codes (kind::i8, s32 acc)
-//                                          or e2m1 codes (kind::f8f6f4, f32 acc)
+//                                          or e2m1 codes (f32 acc: kind::mxf4
+//                                          for CTA pairs, kind::f8f6f4 else)
 //   y[m, n]   = bf16(acc * (xs[m] * gamma[group(n)]))   (or the raw acc)
+//
+// FP4 on CTA pairs runs at the full 4-bit tensor rate through the
+// block-scaled kind::mxf4: A and B are packed e2m1 (two per byte, 128 bytes =
+// 256 k per swizzled row, half the shared-memory bytes of the padded
+// f8f6f4 form), and every ue8m0 block scale is 1.0 (0x7F), written once into
+// tensor memory at start-up, so the products and their fp32 sums are those
+// of the unscaled codes. The scale columns take part of tensor memory, so
+// these tiles are 192 outputs wide (two accumulators of 192 columns + the
+// scales in 512).
 //
 // Persistent, warp-specialised kernel. In the CTA-pair form (two CTAs of a
 // cluster on one TPC, tcgen05 cta_group::2) a pair owns a 256-token x
@@ -39,17 +49,21 @@ constexpr int TMEM_COLS = 512;
 // A TMA instruction costs the issuing thread a few hundred ns whatever its
 // size, so the CTA-pair form moves 256-deep k-blocks (32 KB of activations in
 // one 3-D box) and splits the activation and weight loads over two warps.
-template <bool PAIR>
+// MX: block-scaled FP4 on CTA pairs (packed e2m1 operands, 192-wide tiles).
+template <bool PAIR, bool MX = false>
 struct Layout {
+  static constexpr int BN_T = MX ? 192 : BN;        // output columns per tile
   static constexpr int BK = PAIR ? 256 : 128;       // k-block depth in elements
-  static constexpr int KSUB = BK / 128;             // 128-deep swizzled chunks per k-block
-  static constexpr int S_TMA = PAIR ? 4 : 5;        // activation ring
-  static constexpr int S_W = PAIR ? 2 : 4;          // packed-weight ring
-  static constexpr int S_B = PAIR ? 2 : 3;          // unpacked-weight ring
-  static constexpr int BROWS = PAIR ? BN / 2 : BN;  // weight rows staged per CTA
-  static constexpr int A_BYTES = KSUB * SUB;
+  static constexpr int KSUB = BK / 128;             // 128-deep swizzled chunks per k-block (int8)
+  static constexpr int S_TMA = MX ? 6 : PAIR ? 4 : 5;  // activation ring
+  static constexpr int S_W = MX ? 4 : PAIR ? 2 : 4;    // packed-weight ring
+  static constexpr int S_B = MX ? 3 : PAIR ? 2 : 3;    // unpacked-weight ring
+  static constexpr int BROWS = PAIR ? BN_T / 2 : BN_T;  // weight rows staged per CTA
+  static constexpr int ROW_BYTES = MX ? BK / 2 : BK;    // bytes of one k-block row in smem
+  static constexpr int A_BYTES = MX ? BM * ROW_BYTES : KSUB * SUB;
   static constexpr int WP_BYTES = BROWS * (BK / 4);
-  static constexpr int B_BYTES = BROWS * BK;
+  static constexpr int B_BYTES = BROWS * ROW_BYTES;
+  static constexpr int SF_COL = 2 * BN_T;           // MX: first tensor-memory column of the scales
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + S_TMA * A_BYTES;
   static constexpr int OFF_WP = OFF_B + S_B * B_BYTES;
@@ -79,8 +93,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmW,
                       const __grid_constant__ CUtensorMap tmY, const Params p) {
-  using L = Layout<PAIR>;
+  constexpr bool MX = FP4 && PAIR;
+  using L = Layout<PAIR, MX>;
   constexpr int S_TMA = L::S_TMA, S_W = L::S_W, S_B = L::S_B, BK = L::BK, A_BYTES = L::A_BYTES;
+  constexpr int BN = L::BN_T;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -123,6 +139,24 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (PAIR) cluster_sync();  // peer barriers initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *s_tmem;
+  if constexpr (MX) {
+    // every block scale 1.0: columns SF_COL..511 of all 128 lanes hold 0x7F
+    // bytes (the scales of A at SF_COL, of B at SF_COL + 32), written by the
+    // four epilogue warps (one lane quarter each) before the first MMA
+    if (warp >= 4 && warp < 8) {
+      uint32_t ones[32];
+#pragma unroll
+      for (int i = 0; i < 32; ++i) ones[i] = 0x7F7F7F7Fu;
+      const uint32_t lane_base = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+#pragma unroll
+      for (int c = L::SF_COL; c < TMEM_COLS; c += 32) tmem_st32(lane_base + c, ones);
+      tmem_st_wait();
+      tc_fence_before();
+    }
+    __syncthreads();
+    if (PAIR) cluster_sync();
+    tc_fence_after();
+  }
   // Only now (TMEM held) may the next kernel in the stream start its CTAs.
   pdl_trigger();
 
@@ -138,7 +172,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     *s_abort = 1;
     report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
   };
-  constexpr uint32_t A_TX = FP4 ? L::A_BYTES / 2 : L::A_BYTES;  // global bytes (packed e2m1 = half)
+  // global bytes per activation box (the padded f8f6f4 form reads half of what it stages)
+  constexpr uint32_t A_TX = (FP4 && !MX) ? L::A_BYTES / 2 : L::A_BYTES;
 
   if (warp == 0 || warp == 2) {
     // ----------------------------------------- TMA producers (A: warp 0, W: warp 2)
@@ -157,7 +192,10 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (!mbar_wait(act ? &empty[s] : &wempty[s], ph ^ 1, tmo, s_abort)) { fail(); ok = false; break; }
           if (act) {
             uint8_t* dst = smem + L::OFF_A + s * A_BYTES;
-            if (PAIR) {
+            if (MX) {  // packed e2m1 rows: one 128-byte (256 k) box column per k-block
+              if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
+              tma_load_2d_pair(dst, &tmA, lead(&afull[s]), kb * (BK / 2), m0);
+            } else if (PAIR) {
               if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
               tma_load_3d_pair(dst, &tmA, lead(&afull[s]), 0, m0, kb * L::KSUB);
             } else {
@@ -185,7 +223,10 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   } else if (warp == 1) {
     // -------------------------------------------------------- MMA issuer
     if (lane == 0 && leader) {
-      constexpr uint32_t idesc = FP4 ? make_idesc(1, 5, 5, TILE_M, BN) : make_idesc(2, 1, 1, TILE_M, BN);
+      constexpr uint32_t idesc = MX    ? make_idesc_mxf4(TILE_M, BN)
+                                 : FP4 ? make_idesc(1, 5, 5, TILE_M, BN)
+                                       : make_idesc(2, 1, 1, TILE_M, BN);
+      const uint32_t sfa = tmem_base + L::SF_COL, sfb = tmem_base + L::SF_COL + 32;
       uint32_t it = 0, tl = 0;
       bool ok = true;
       for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride, ++tl) {
@@ -202,6 +243,14 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                                  : mbar_wait(&bfull[b], bph, tmo, s_abort));
           if (!got) { fail(); ok = false; break; }
           tc_fence_after();
+          if constexpr (MX) {
+            // 4 MMAs of K = 64 (32 bytes of packed e2m1) along the 128-byte rows
+            const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES);
+            const uint64_t bdesc = smem_desc_sw128(sB + b * L::B_BYTES);
+#pragma unroll
+            for (int kk = 0; kk < BK / 64; ++kk)
+              mma_mxf4_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb, (kb | kk) != 0);
+          } else
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
             // chunk kk / 4 of the k-block; advance 32 bytes (2 x 16 B) along K
@@ -361,6 +410,20 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t src = sW + s * L::WP_BYTES;
         const uint32_t dst = sB + b * L::B_BYTES;
         constexpr int WPR = BK / 16;  // packed words per weight row
+        if constexpr (MX) {
+          // two packed words (32 k) -> one 16-byte group of 32 e2m1 nibbles
+          // (even k low), chunk c of the row's 128-byte swizzled line
+#pragma unroll
+          for (int i = 0; i < (L::BROWS * 8) / 256; ++i) {
+            const int g = ut + 256 * i;
+            const int n = g >> 3, c = g & 7;
+            const uint32_t w0 = ld_shared_u32(src + n * (BK / 4) + 8 * c);
+            const uint32_t w1 = ld_shared_u32(src + n * (BK / 4) + 8 * c + 4);
+            const uint32_t addr = dst + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
+            st_shared_v4(addr, codes_to_e2m1(codes_lo(w0)), codes_to_e2m1(codes_hi(w0)),
+                         codes_to_e2m1(codes_lo(w1)), codes_to_e2m1(codes_hi(w1)));
+          }
+        } else
 #pragma unroll
         for (int i = 0; i < (L::BROWS * WPR) / 256; ++i) {
           const int w = ut + 256 * i;          // packed word index in the tile
@@ -429,11 +492,12 @@ template <bool FP4, bool PAIR>
 static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const CUtensorMap& tmY,
                             const gemm::Params& p, cudaStream_t s) {
   using namespace gemm;
+  using L = Layout<PAIR, FP4 && PAIR>;
   auto kern = bitlinear_gemm_kernel<FP4, PAIR>;
   static bool attr_set = false;  // once per process (not during graph capture)
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         Layout<PAIR>::SMEM_BYTES);
+                                         L::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -441,10 +505,10 @@ static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, cons
   if (PAIR) {
     const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;
     return launch_kernel(kern, dim3(static_cast<unsigned>(2 * pairs)), dim3(THREADS),
-                         Layout<PAIR>::SMEM_BYTES, s, 2u, tmA, tmW, tmY, p);
+                         L::SMEM_BYTES, s, 2u, tmA, tmW, tmY, p);
   }
   return launch_kernel(kern, dim3(static_cast<unsigned>(p.num_tiles < sms ? p.num_tiles : sms)),
-                       dim3(THREADS), Layout<PAIR>::SMEM_BYTES, s, 0u, tmA, tmW, tmY, p);
+                       dim3(THREADS), L::SMEM_BYTES, s, 0u, tmA, tmW, tmY, p);
 }
 
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why) {
@@ -452,13 +516,20 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   // CTA pairs once there are two 128-row halves to fill; their 3-D activation
   // view needs whole 128-deep K chunks
   const bool pair = a.M > BM && a.K % 128 == 0;
-  const int brows = pair ? BN / 2 : BN;
+  const bool mx = pair && fp4;  // block-scaled FP4 on packed operands
+  const int bn = mx ? Layout<true, true>::BN_T : BN;
+  const int brows = pair ? bn / 2 : bn;
   const int BK = pair ? Layout<true>::BK : Layout<false>::BK;
   CUtensorMap tmA, tmW, tmY;
   cudaError_t e;
   const CUtensorMapDataType adt = fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t row_bytes = fp4 ? a.K / 2 : a.K;
-  if (pair) {
+  if (mx) {
+    // packed e2m1 codes as bytes [M][K/2]: 128 rows x 128 bytes (256 k) per
+    // box, 128-byte swizzle; a ragged last k-block reads zeros past K
+    e = make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, a.K / 2, a.M, row_bytes, BK / 2, BM,
+                    CU_TENSOR_MAP_SWIZZLE_128B, why);
+  } else if (pair) {
     // [K/128 chunks][M rows][128 elements]: one box = 2 chunks x 128 rows,
     // i.e. two standard 128-byte-swizzled 128 x 128 tiles back to back
     const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.M), static_cast<cuuint64_t>(a.K / 128)};
@@ -488,7 +559,7 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.num_kb = static_cast<int>((a.K + BK - 1) / BK);
   const int tile_m = pair ? 2 * BM : BM;
   p.tiles_m = static_cast<int>((a.M + tile_m - 1) / tile_m);
-  const int tiles_n = static_cast<int>((a.N + BN - 1) / BN);
+  const int tiles_n = static_cast<int>((a.N + bn - 1) / bn);
   p.num_tiles = p.tiles_m * tiles_n;
   p.xs = a.xs;
   p.gamma = a.gamma;

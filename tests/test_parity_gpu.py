@@ -73,7 +73,7 @@ def test_fp4_rounding_midpoints():
     vals = []
     for m in mids:
         b = O.f32_to_bf16(np.float32(m))
-        vals += [m, float(O.bf16_to_f32(b + 1)[()]), float(O.bf16_to_f32(b - 1)[()])]
+        vals += [m, float(np.ravel(O.bf16_to_f32(b + 1))[0]), float(np.ravel(O.bf16_to_f32(b - 1))[0])]
     vals += [0.0, -0.0, 0.1, -0.1, 6.0, 4.0, 3.0]
     vals += [-v for v in vals]
     row = np.array(vals + [0.0] * (-len(vals) % 16), np.float32)
@@ -137,7 +137,7 @@ def prep_weights(K, N, groups, seed):
 
 GEMM_SHAPES = [  # (M, N, K): single tile, ragged M/N, half k-block, many tiles
     (16, 256, 256), (1, 16, 64), (130, 272, 320), (257, 512, 1024), (2048, 4096, 256),
-    (300, 768, 2048 + 64)]
+    (300, 768, 2048 + 64), (384, 400, 384)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
