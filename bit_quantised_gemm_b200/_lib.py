@@ -53,6 +53,7 @@ _SIGS = {
     "bitlinear_gemv_w2_quant": ([_P, _P, _I64, _INT, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P],
                                 _INT),
     "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
+    "kv_keep4_positions": ([_P, _I64, _P, _INT, _P, _P, _P], _INT),
     "bitlinear_check_status": ([_P, _P], _INT),
     "bitlinear_debug_wait_timeout": ([_P, _I64, _P], _INT),
 }
@@ -279,6 +280,22 @@ def kv_quant_3bit(kv: torch.Tensor, keep4_pos: torch.Tensor | None, codes3=None,
     _check(lib().kv_quant_3bit(_ptr(kv), T, H, D, _ptr(keep4_pos), n4, _ptr(codes3), _ptr(codes4),
                                _ptr(scale), _stream(stream)))
     return codes3, codes4, scale
+
+
+def kv_keep4_positions(token_ids: torch.Tensor, special_ids, stream=None) -> torch.Tensor:
+    """Sorted positions t with token_ids[t] in special_ids (e.g. bos and eos),
+    the 4-bit list of kv_quant_3bit; the count is read back to size it."""
+    _require_cuda(token_ids)
+    if token_ids.dtype != torch.int32 or token_ids.dim() != 1 or not token_ids.is_contiguous():
+        raise ValueError("token_ids must be a contiguous 1-D int32 tensor")
+    sp = (_c.c_int32 * len(special_ids))(*[int(v) for v in special_ids])
+    T = token_ids.numel()
+    pos = torch.empty(max(T, 1), dtype=torch.int32, device=token_ids.device)
+    count = torch.zeros(1, dtype=torch.int32, device=token_ids.device)
+    _check(lib().kv_keep4_positions(_ptr(token_ids), T, _c.addressof(sp), len(special_ids), _ptr(pos),
+                                    _ptr(count), _stream(stream)))
+    (stream or torch.cuda.current_stream(token_ids.device)).synchronize()
+    return pos[:int(count.item())]
 
 
 def kv_attention_3bit(q: torch.Tensor, k_store, v_store, keep4_pos: torch.Tensor | None, out=None,

@@ -131,7 +131,7 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 103; }
+int bitlinear_version(void) { return 104; }
 
 int bitlinear_set_launch_overlap(int enable) {
   g_overlap.store(enable != 0);
@@ -341,6 +341,19 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
     return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: T * H * D / 8 must stay below 2^32");
   cudaError_t e = blt::launch_kv_quant(kv, T, H, D, keep4_pos, n_keep4, codes3, codes4, scale, stream);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_quant_3bit launch");
+}
+
+int kv_keep4_positions(const int32_t* token_ids, int64_t T, const int32_t* special_ids,
+                       int n_special, int32_t* pos_out, int32_t* count_out,
+                       bitlinear_stream_t stream) {
+  if (T < 0 || T > 0x7FFFFFFF) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_keep4_positions: bad T");
+  if (n_special < 1 || n_special > 8 || !special_ids)
+    return fail(BITLINEAR_ERR_INVALID_ARG, "kv_keep4_positions: 1 to 8 special ids");
+  if (!count_out || (T > 0 && (!token_ids || !pos_out)))
+    return fail(BITLINEAR_ERR_INVALID_ARG, "kv_keep4_positions: null pointer");
+  cudaError_t e = blt::launch_keep4_positions(token_ids, T, special_ids, n_special, pos_out, count_out,
+                                              stream);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "kv_keep4_positions launch");
 }
 
 int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,

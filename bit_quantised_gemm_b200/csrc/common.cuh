@@ -71,19 +71,23 @@ __device__ __forceinline__ uint4 unpack16_s8(uint32_t w) {
   return o;
 }
 
-// One nibble per code -> e2m1 nibble: code 0 -> 0xA (-1.0), 1 -> 0x0, 2 -> 0x2 (+1.0).
-__device__ __forceinline__ uint32_t codes_to_e2m1(uint32_t x) {
-  const uint32_t nz = ~x & 0x11111111u;                 // code is 0 or 2: weight non-zero
-  const uint32_t neg = ~x & ~(x >> 1) & 0x11111111u;    // code is 0: weight -1
-  return (nz << 1) | (neg << 3);
+// 16 weights -> two words of 8 e2m1 nibbles each (elements 0-7 and 8-15,
+// even k in the low nibble): code 0 -> 0xA (-1.0), 1 -> 0x0, 2 -> 0x2 (+1.0).
+// Eight logic ops: for the code bits (c1 c0) of element 8h + i, nibble i of
+// the result gets bit 1 = !c0 (a non-zero weight) and bit 3 = !c0 & !c1
+// (weight -1). For h = 0 those bits sit 1 and 3 places above c0 and 2 above
+// c1; for h = 1, 1 below and 1 above c0 and at c1 itself.
+__device__ __forceinline__ void e2m1_words(uint32_t w, uint32_t& lo, uint32_t& hi) {
+  const uint32_t t1 = w << 1, t2 = w << 2, t3 = w << 3, r1 = w >> 1;
+  lo = (~t1 & 0x22222222u) | (~t3 & ~t2 & 0x88888888u);
+  hi = (~r1 & 0x22222222u) | (~t1 & ~w & 0x88888888u);
 }
 
 // 16 weights -> one 16-byte e2m1 group in the padded shared-memory form the
 // f8f6f4 MMA reads: 16 nibbles (even k low) in the first 8 bytes, 8 zero bytes.
 __device__ __forceinline__ uint4 unpack16_e2m1(uint32_t w) {
   uint4 o;
-  o.x = codes_to_e2m1(codes_lo(w));
-  o.y = codes_to_e2m1(codes_hi(w));
+  e2m1_words(w, o.x, o.y);
   o.z = 0u;
   o.w = 0u;
   return o;

@@ -411,29 +411,41 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const uint32_t dst = sB + b * L::B_BYTES;
         constexpr int WPR = BK / 16;  // packed words per weight row
         if constexpr (MX) {
+          // all of a thread's packed words are loaded before its first store
+          // (the ordered shared-memory accesses would otherwise serialise
+          // the iterations)
           // two packed words (32 k) -> one 16-byte group of 32 e2m1 nibbles
           // (even k low), chunk c of the row's 128-byte swizzled line
+          constexpr int NI = (L::BROWS * 8) / 256;
+          uint2 wv[NI];
 #pragma unroll
-          for (int i = 0; i < (L::BROWS * 8) / 256; ++i) {
+          for (int i = 0; i < NI; ++i) {
+            const int g = ut + 256 * i;
+            wv[i] = ld_shared_v2(src + (g >> 3) * (BK / 4) + 8 * (g & 7));
+          }
+#pragma unroll
+          for (int i = 0; i < NI; ++i) {
             const int g = ut + 256 * i;
             const int n = g >> 3, c = g & 7;
-            const uint32_t w0 = ld_shared_u32(src + n * (BK / 4) + 8 * c);
-            const uint32_t w1 = ld_shared_u32(src + n * (BK / 4) + 8 * c + 4);
-            const uint32_t addr = dst + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4);
-            st_shared_v4(addr, codes_to_e2m1(codes_lo(w0)), codes_to_e2m1(codes_hi(w0)),
-                         codes_to_e2m1(codes_lo(w1)), codes_to_e2m1(codes_hi(w1)));
+            uint4 o;
+            e2m1_words(wv[i].x, o.x, o.y);
+            e2m1_words(wv[i].y, o.z, o.w);
+            st_shared_v4(dst + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4), o.x, o.y, o.z, o.w);
           }
-        } else
+        } else {
+          // one word at a time: with the shared-memory port saturated by the
+          // MMA and TMA traffic, batching the loads was not faster here
 #pragma unroll
-        for (int i = 0; i < (L::BROWS * WPR) / 256; ++i) {
-          const int w = ut + 256 * i;          // packed word index in the tile
-          const int n = w / WPR, j = w % WPR;  // row, 16-deep K group
-          const int sub = j >> 3, c = j & 7;   // 128-deep chunk, 16-byte column in it
-          const uint32_t word = ld_shared_u32(src + 4 * w);
-          const uint4 o = FP4 ? unpack16_e2m1(word) : unpack16_s8(word);
-          const uint32_t addr = dst + sub * (L::BROWS * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
-                                ((c ^ (n & 7)) << 4);
-          st_shared_v4(addr, o.x, o.y, o.z, o.w);
+          for (int i = 0; i < (L::BROWS * WPR) / 256; ++i) {
+            const int w = ut + 256 * i;          // packed word index in the tile
+            const int n = w / WPR, j = w % WPR;  // row, 16-deep K group
+            const int sub = j >> 3, c = j & 7;   // 128-deep chunk, 16-byte column in it
+            const uint32_t word = ld_shared_u32(src + 4 * w);
+            const uint4 o = FP4 ? unpack16_e2m1(word) : unpack16_s8(word);
+            const uint32_t addr = dst + sub * (L::BROWS * 128) + (n >> 3) * 1024 + (n & 7) * 128 +
+                                  ((c ^ (n & 7)) << 4);
+            st_shared_v4(addr, o.x, o.y, o.z, o.w);
+          }
         }
         fence_proxy_async_smem();  // each thread's smem writes -> async proxy
         __syncwarp();

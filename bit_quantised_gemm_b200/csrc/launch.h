@@ -17,6 +17,8 @@ cudaError_t launch_kv_attention(const uint16_t* q, int64_t B, int64_t H, int64_t
                                 const uint8_t* v3, const uint8_t* v4, const float* vs,
                                 const int32_t* keep4, int64_t n4, uint16_t* out, int* status,
                                 uint64_t timeout_ns, cudaStream_t s, const char** why);
+cudaError_t launch_keep4_positions(const int32_t* ids, int64_t T, const int32_t* special, int n_special,
+                                   int32_t* pos, int32_t* count, cudaStream_t s);
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s);

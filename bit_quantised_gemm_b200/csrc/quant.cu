@@ -469,6 +469,57 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
   }
 }
 
+// ------------------------------------------------ 4-bit token positions
+// One block walks the token ids in chunks of 256 x 4: each thread tests its
+// 4 consecutive ids against the special ids, a block prefix sum of the
+// matches gives every thread its output offset, and the running total moves
+// on to the next chunk, so the positions come out in increasing order.
+struct SpecialIds {
+  int32_t id[8];
+  int n;
+};
+
+__global__ void __launch_bounds__(kQuantThreads) keep4_positions_kernel(
+    const int32_t* __restrict__ ids, int64_t T, SpecialIds sp, int32_t* __restrict__ pos,
+    int32_t* __restrict__ count) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ uint32_t sums[8];
+  uint32_t total = 0;
+  for (int64_t base = 0; base < T; base += 4 * kQuantThreads) {
+    const int64_t t0 = base + 4 * static_cast<int64_t>(threadIdx.x);
+    uint32_t hit = 0u, n = 0u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      bool m = false;
+      if (t0 + i < T) {
+        const int32_t v = __ldg(ids + t0 + i);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) m |= (j < sp.n && v == sp.id[j]);
+      }
+      hit |= (m ? 1u : 0u) << i;
+      n += m ? 1u : 0u;
+    }
+    const uint32_t incl = block_scan_256(n, sums);
+    uint32_t o = total + incl - n;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+      if ((hit >> i) & 1u) pos[o++] = static_cast<int32_t>(t0 + i);
+    total += sums[kQuantThreads / 32 - 1];  // the chunk's matches
+    __syncthreads();                         // sums is rewritten by the next chunk
+  }
+  if (threadIdx.x == 0) *count = static_cast<int32_t>(total);
+}
+
+cudaError_t launch_keep4_positions(const int32_t* ids, int64_t T, const int32_t* special, int n_special,
+                                   int32_t* pos, int32_t* count, cudaStream_t s) {
+  SpecialIds sp{};
+  for (int j = 0; j < n_special; ++j) sp.id[j] = special[j];
+  sp.n = n_special;
+  return launch_kernel(keep4_positions_kernel, dim3(1), dim3(kQuantThreads), 0, s, 0u, ids, T, sp,
+                       pos, count);
+}
+
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s) {

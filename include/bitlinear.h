@@ -200,6 +200,23 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
                   bitlinear_stream_t stream);
 
 /*
+ * The positions kept at 4 bits, from the token ids ([R] "Эксперименты": the
+ * <bos> and <eos> tokens stay at 4 bits): every t < T whose token_ids[t]
+ * equals one of special_ids, in increasing order; the list kv_quant_3bit and
+ * kv_attention_3bit take.
+ *   token_ids    device int32 [T]
+ *   special_ids  host int32 [n_special], 1 <= n_special <= 8 (e.g. the bos
+ *                and eos ids)
+ *   pos_out      device int32 [T]; the first *count_out entries are written
+ *   count_out    device int32 [1]
+ * Runs as one block on the stream (the count is device memory: read it back
+ * to size the list on the host).
+ */
+int kv_keep4_positions(const int32_t* token_ids, int64_t T, const int32_t* special_ids,
+                       int n_special, int32_t* pos_out, int32_t* count_out,
+                       bitlinear_stream_t stream);
+
+/*
  * Decode attention over that cache ([R] "Эксперименты": the 3-bit KV cache
  * with <bos>/<eos> at 4 bits is what attention reads at inference). For
  * every query (b, h) and every cached token t < T of head h:

@@ -54,7 +54,8 @@ CUDA library implements from its own code) are:
      clamp(rne(x * (Q / a')), -4, 3), stored as code + 4 in a little-endian
      3-bit stream (code d in bits [3d, 3d+3)); tokens listed in keep4_pos use
      Q = 7, clamp [-8, 7], stored as code + 8, two per byte, low nibble first;
-     their 3-bit row is all zero bytes. scale = a' / Q.
+     their 3-bit row is all zero bytes. scale = a' / Q. The listed tokens are
+     those whose id is one of the special ids (bos, eos), in position order.
   C10 decode attention over that cache (the pages name only its storage
      precision): softmax((q . k_t) / sqrt(D)) over every cached token t of
      the query's head, weights applied to the dequantised v_t; fp64 here.
@@ -338,6 +339,16 @@ def bitlinear_fp4(xf4_packed, xs, Wt, gamma, group_ends):
 
 
 # -------------------------------------------------------------- C9 KV cache
+def keep4_positions(token_ids, special_ids):
+    """C9: the positions whose token id is one of special_ids (the bos and eos
+    ids), in increasing order, as int32."""
+    ids = np.asarray(token_ids, dtype=np.int64)
+    hit = np.zeros(ids.shape, dtype=bool)
+    for v in special_ids:
+        hit |= ids == int(v)
+    return np.flatnonzero(hit).astype(np.int32)
+
+
 def kv_quant_3bit(kv_bits: np.ndarray, keep4_pos=(0,)):
     """C9 per (token, head) KV quantiser.
 

@@ -20,7 +20,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(_lib._SIGS)
-    assert B.version() == 103
+    assert B.version() == 104
 
 
 @pytest.mark.parametrize("K,N,groups,seed", [
@@ -124,6 +124,19 @@ def test_kv_attention_argument_errors():
     assert call(q=None) == _lib.ERR_INVALID_ARG
     assert call(out=FAKE + 2) == _lib.ERR_ALIGNMENT
     assert call(B=0) == _lib.OK
+
+
+def test_keep4_positions_argument_errors():
+    L = B.lib()
+    sp = (ctypes.c_int32 * 2)(1, 2)
+    many = (ctypes.c_int32 * 9)(*range(9))
+    addr = ctypes.addressof
+    assert L.kv_keep4_positions(FAKE, 16, addr(sp), 0, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_keep4_positions(FAKE, 16, addr(many), 9, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_keep4_positions(FAKE, 16, None, 2, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_keep4_positions(FAKE, -1, addr(sp), 2, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_keep4_positions(None, 16, addr(sp), 2, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
+    assert L.kv_keep4_positions(FAKE, 16, addr(sp), 2, FAKE, None, None) == _lib.ERR_INVALID_ARG
 
 
 def test_quantiser_argument_errors():

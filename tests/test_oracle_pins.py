@@ -312,6 +312,17 @@ def test_kv_golden():
     assert s[0, 0] == np.float32(3) / np.float32(7)
 
 
+def test_keep4_positions_golden():
+    g = golden("keep4_ids.txt")
+    ids = np.array([int(v) for v in g["ids"]], np.int32)
+    got = O.keep4_positions(ids, [int(v) for v in g["special"]])
+    assert got.dtype == np.int32 and got.tolist() == [int(v) for v in g["positions"]]
+    got = O.keep4_positions(ids, [int(v) for v in g["special_bos"]])
+    assert got.tolist() == [int(v) for v in g["positions_bos"]]
+    assert O.keep4_positions(np.zeros(0, np.int32), [1]).size == 0
+    assert O.keep4_positions(ids, [99]).size == 0
+
+
 def test_kv_invariants_and_roundtrip():
     rng = np.random.default_rng(13)
     T, H, D = 20, 4, 128

@@ -111,6 +111,37 @@ def test_topk_full_size_o_proj():
     assert np.array_equal(host(mask), O.pack_mask_bits(m_o))
 
 
+@pytest.mark.parametrize("T,special,p", [(0, (1,), 0.0), (1, (1, 2), 1.0), (9, (1, 2), 0.3),
+                                         (1024, (1, 2), 0.01), (5000, (7,), 0.5), (70000, (1, 2), 0.002),
+                                         (3000, (1, 2), 0.0), (2049, (3, 1, 2, 9), 1.0)])
+def test_keep4_positions_parity(T, special, p):
+    """Token ids -> the sorted positions kept at 4 bits (bit-exact), several
+    1024-id chunks, ragged tails, none and all matching."""
+    rng = np.random.default_rng(T + len(special))
+    ids = rng.integers(10, 32000, size=T).astype(np.int32)
+    hit = rng.random(T) < p
+    ids[hit] = rng.choice(np.array(special, np.int32), size=int(hit.sum()))
+    got = B.kv_keep4_positions(torch.from_numpy(ids).to(DEV), special)
+    assert np.array_equal(host(got), O.keep4_positions(ids, special))
+
+
+def test_kv_quant_with_positions_from_token_ids():
+    """bos / eos ids -> positions -> the 3-bit cache, against the oracle's."""
+    rng = np.random.default_rng(3)
+    T, H, D = 300, 4, 128
+    ids = rng.integers(3, 32000, size=T).astype(np.int32)
+    ids[[0, 120, 121]] = 1
+    ids[[119, 299]] = 2
+    kv = W.normal_bf16(rng, (T, H, D))
+    pos = B.kv_keep4_positions(torch.from_numpy(ids).to(DEV), (1, 2))
+    keep = O.keep4_positions(ids, (1, 2))
+    assert np.array_equal(host(pos), keep)
+    c3, c4, s = B.kv_quant_3bit(dev_bf16(kv), pos)
+    c3_o, c4_o, s_o = O.kv_quant_3bit(kv, tuple(keep))
+    assert np.array_equal(host(c3), c3_o) and np.array_equal(host(c4), c4_o)
+    assert np.array_equal(host(s), s_o)
+
+
 @pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("keep", [(0,), (0, 5, 6, 37), ()])
 def test_kv_quant_parity(D, keep):
