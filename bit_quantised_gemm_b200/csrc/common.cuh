@@ -22,8 +22,15 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 }
 
 // Integer code of one activation: clamp(rne(h * inv), lo, hi), fp32 multiply.
+// The rounding runs on the FMA pipe rather than the quarter-rate conversion
+// unit: for |v| < 2^22, v + 1.5 * 2^23 rounds v to the nearest integer (ties
+// to even) and that integer is the low bits of the sum. Every caller has
+// |h * inv| <= Q (1 + 2^-23) with Q <= 127 (|h| never exceeds the absmax
+// its scale comes from).
 __device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi) {
-  return static_cast<int>(fminf(fmaxf(rintf(__fmul_rn(h, inv)), lo), hi));
+  const float r = __fadd_rn(__fmul_rn(h, inv), 12582912.f);
+  const int c = __float_as_int(r) - 0x4B400000;
+  return min(max(c, static_cast<int>(lo)), static_cast<int>(hi));
 }
 
 __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
