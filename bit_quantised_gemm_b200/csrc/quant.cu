@@ -245,18 +245,23 @@ cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, i
 }
 
 // ----------------------------------------------------------------- top-k
-// One block per row; thread t owns the contiguous elements [t*E, t*E+E).
-// Radix select on the 15-bit |bf16| key: an 8-bit histogram of key >> 7,
-// then a 7-bit histogram of the low bits inside the selected bin, gives the
-// threshold key T and the count of keys above it. Keys equal to T are kept
-// in column order until k are kept (a block prefix sum gives each thread's
-// starting rank among the equal keys).
+// One block per row; thread t owns the contiguous elements [t*E, t*E+E),
+// held as packed bf16 pairs. Radix select on the 15-bit |bf16| key: an 8-bit
+// histogram of key >> 7, then a 7-bit histogram of the low bits inside the
+// selected bin, gives the threshold key T and the count of keys above it.
+// Keys equal to T are kept in column order until k are kept (a block prefix
+// sum gives each thread's starting rank among the equal keys).
+// Columns past K are read as key 0: they come after every real column in
+// the (key descending, column ascending) order, so they are never among the
+// k kept and the loops need no bounds tests.
 template <int E>
 __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
     const uint16_t* __restrict__ x, int K, int64_t ldx, int k, int8_t* __restrict__ q_out,
     float* __restrict__ xs_out, uint8_t* __restrict__ mask_out) {
   pdl_wait();  // inputs come from the previous kernel in the stream
   pdl_trigger();
+  static_assert(E % 8 == 0, "whole 16-byte groups");
+  constexpr int NW = E / 2;  // packed pairs per thread
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sums[8];
   __shared__ float red[8];
@@ -266,25 +271,24 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   const int base = t * E;
   const int nvalid = max(0, min(E, K - base));  // multiple of 8
 
-  uint16_t v[E];
+  uint32_t w[NW];
 #pragma unroll
   for (int c = 0; c < E / 8; ++c) {
-    uint4 w = make_uint4(0, 0, 0, 0);
-    if (c * 8 < nvalid) w = __ldg(reinterpret_cast<const uint4*>(x + m * ldx + base) + c);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      v[c * 8 + 2 * i] = static_cast<uint16_t>(ws[i] & 0xFFFFu);
-      v[c * 8 + 2 * i + 1] = static_cast<uint16_t>(ws[i] >> 16);
-    }
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (c * 8 < nvalid) u = __ldg(reinterpret_cast<const uint4*>(x + m * ldx + base) + c);
+    w[4 * c] = u.x; w[4 * c + 1] = u.y; w[4 * c + 2] = u.z; w[4 * c + 3] = u.w;
   }
+  auto key_lo = [](uint32_t v) { return v & 0x7FFFu; };
+  auto key_hi = [](uint32_t v) { return (v >> 16) & 0x7FFFu; };
 
   // pass 1: high 8 bits of the key
   hist[t] = 0u;
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < E; ++i)
-    if (i < nvalid) atomicAdd(&hist[(v[i] & 0x7FFF) >> 7], 1u);
+  for (int j = 0; j < NW; ++j) {
+    atomicAdd(&hist[(w[j] >> 7) & 0xFFu], 1u);
+    atomicAdd(&hist[(w[j] >> 23) & 0xFFu], 1u);
+  }
   __syncthreads();
   {
     const uint32_t c = hist[255 - t];
@@ -302,9 +306,10 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   hist[t] = 0u;
   __syncthreads();
 #pragma unroll
-  for (int i = 0; i < E; ++i) {
-    const uint32_t key = v[i] & 0x7FFF;
-    if (i < nvalid && (key >> 7) == b1) atomicAdd(&hist[key & 127], 1u);
+  for (int j = 0; j < NW; ++j) {
+    const uint32_t lo = key_lo(w[j]), hi = key_hi(w[j]);
+    if ((lo >> 7) == b1) atomicAdd(&hist[lo & 127u], 1u);
+    if ((hi >> 7) == b1) atomicAdd(&hist[hi & 127u], 1u);
   }
   __syncthreads();
   {
@@ -320,30 +325,33 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   const uint32_t T = (b1 << 7) | sel[0];
   const uint32_t need_eq = static_cast<uint32_t>(k) - above1 - sel[1];  // >= 1
 
-  // pass 3: rank of equal keys in column order
-  uint32_t n_eq = 0;
-#pragma unroll
-  for (int i = 0; i < E; ++i) n_eq += (i < nvalid && (v[i] & 0x7FFF) == T) ? 1u : 0u;
-  uint32_t rank = block_scan_256(n_eq, sums) - n_eq;  // exclusive prefix
-
-  uint32_t keep_bits[(E + 31) / 32];
-#pragma unroll
-  for (int j = 0; j < (E + 31) / 32; ++j) keep_bits[j] = 0u;
-  float amax = 0.f;
+  // keys above T are kept; keys equal to T are kept in column order until
+  // k are kept (the block prefix of their counts ranks this thread's)
+  static_assert(E <= 64, "bit masks of 64 bits");
+  uint64_t gt = 0u, eq = 0u;
+  uint32_t kmax = 0u;  // the row's largest key: the largest kept one (k >= 1 here)
 #pragma unroll
   for (int i = 0; i < E; ++i) {
-    const uint32_t key = v[i] & 0x7FFF;
-    bool keep = false;
-    if (i < nvalid) {
-      if (key > T) keep = true;
-      else if (key == T) { keep = rank < need_eq; ++rank; }
-    }
-    if (keep) {
-      keep_bits[i >> 5] |= 1u << (i & 31);
-      amax = fmaxf(amax, fabsf(__uint_as_float(static_cast<uint32_t>(v[i]) << 16)));
+    const uint32_t key = (i & 1) ? key_hi(w[i >> 1]) : key_lo(w[i >> 1]);
+    gt |= static_cast<uint64_t>(key > T ? 1u : 0u) << i;
+    eq |= static_cast<uint64_t>(key == T ? 1u : 0u) << i;
+    kmax = max(kmax, key);
+  }
+  const uint32_t n_eq = static_cast<uint32_t>(__popcll(eq));
+  const uint32_t rank = block_scan_256(n_eq, sums) - n_eq;  // equal keys in earlier threads
+  uint64_t keep = gt;
+  if (eq) {  // rare: this thread holds keys equal to T; keep its first ones
+    const uint32_t take = rank < need_eq ? min(need_eq - rank, n_eq) : 0u;
+    uint64_t e = eq;
+    for (uint32_t j = 0; j < take; ++j) {
+      keep |= e & (~e + 1u);  // lowest set bit
+      e &= e - 1u;
     }
   }
-  amax = block_max_256(amax, red);
+  uint32_t keep_bits[(E + 31) / 32];
+#pragma unroll
+  for (int j = 0; j < (E + 31) / 32; ++j) keep_bits[j] = static_cast<uint32_t>(keep >> (32 * j));
+  const float amax = block_max_256(__uint_as_float(kmax << 16), red);
   const float a = fmaxf(amax, kEps);
   const float inv = __fdiv_rn(127.f, a);
   if (t == 0) xs_out[m] = __fdiv_rn(a, 127.f);
@@ -351,19 +359,17 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
 #pragma unroll
   for (int c = 0; c < E / 8; ++c) {
     if (c * 8 < nvalid) {
+      const uint32_t kb = keep_bits[(8 * c) >> 5] >> ((8 * c) & 31);  // this group's 8 bits
       int q[8];
-      uint32_t mb = 0u;
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
-        const int idx = c * 8 + i;
-        const bool kp = (keep_bits[idx >> 5] >> (idx & 31)) & 1u;
-        const float xv = __uint_as_float(static_cast<uint32_t>(v[idx]) << 16);
-        q[i] = kp ? quant_code(xv, inv, -128.f, 127.f) : 0;
-        mb |= (kp ? 1u : 0u) << i;
+        const uint32_t v = w[4 * c + (i >> 1)];
+        const float xv = __uint_as_float((i & 1) ? (v & 0xFFFF0000u) : (v << 16));
+        q[i] = ((kb >> i) & 1u) ? quant_code(xv, inv, -128.f, 127.f) : 0;
       }
       reinterpret_cast<uint2*>(q_out + m * K + base)[c] =
           make_uint2(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]));
-      if (mask_out) mask_out[m * (K >> 3) + (base >> 3) + c] = static_cast<uint8_t>(mb);
+      if (mask_out) mask_out[m * (K >> 3) + (base >> 3) + c] = static_cast<uint8_t>(kb & 0xFFu);
     }
   }
 }
