@@ -245,23 +245,66 @@ cudaError_t launch_quant_act(const uint16_t* x, const uint16_t* up, int64_t M, i
 }
 
 // ----------------------------------------------------------------- top-k
-// One block per row; thread t owns the contiguous elements [t*E, t*E+E),
-// held as packed bf16 pairs. Radix select on the 15-bit |bf16| key: an 8-bit
-// histogram of key >> 7, then a 7-bit histogram of the low bits inside the
-// selected bin, gives the threshold key T and the count of keys above it.
-// Keys equal to T are kept in column order until k are kept (a block prefix
-// sum gives each thread's starting rank among the equal keys).
-// Columns past K are read as key 0: they come after every real column in
-// the (key descending, column ascending) order, so they are never among the
-// k kept and the loops need no bounds tests.
-template <int E>
-__global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
+// Inclusive prefix sum over the NT threads of the block (NT / 32 <= 8 warps).
+template <int NT>
+__device__ __forceinline__ uint32_t block_scan(uint32_t v, uint32_t* sums /*[8]*/) {
+  constexpr int NWARP = NT / 32;
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t n = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += n;
+  }
+  if (lane == 31) sums[wid] = v;
+  __syncthreads();
+  if (wid == 0) {
+    uint32_t s = lane < NWARP ? sums[lane] : 0u;
+#pragma unroll
+    for (int o = 1; o < NWARP; o <<= 1) {
+      const uint32_t n = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += n;
+    }
+    if (lane < NWARP) sums[lane] = s;
+  }
+  __syncthreads();
+  if (wid > 0) v += sums[wid - 1];
+  __syncthreads();
+  return v;
+}
+
+template <int NT>
+__device__ __forceinline__ float block_max(float v, float* red /*[8]*/) {
+  v = warp_max(v);
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  if (lane == 0) red[wid] = v;
+  __syncthreads();
+  float r = red[0];
+#pragma unroll
+  for (int i = 1; i < NT / 32; ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+// One block of NT threads per row; thread t owns the contiguous elements
+// [t*E, t*E+E), held as packed bf16 pairs. Radix select on the 15-bit |bf16|
+// key: a 256-bin histogram of key >> 7, then a 128-bin histogram of the low
+// bits inside the selected bin, gives the threshold key T and the count of
+// keys above it. Keys equal to T are kept in column order until k are kept
+// (a block prefix sum of their counts ranks each thread's). Columns past K
+// are read as key 0: they come after every real column in the (key
+// descending, column ascending) order, so they are never among the k kept
+// and the loops need no bounds tests. The per-row work outside the element
+// loops (scans, barriers) is the same for any E, so rows of 4096 use 128
+// threads of 32 elements.
+template <int NT, int E>
+__global__ void __launch_bounds__(NT, (E >= 32 ? 1024 : 2048) / NT) topk_i8_kernel(
     const uint16_t* __restrict__ x, int K, int64_t ldx, int k, int8_t* __restrict__ q_out,
     float* __restrict__ xs_out, uint8_t* __restrict__ mask_out) {
   pdl_wait();  // inputs come from the previous kernel in the stream
   pdl_trigger();
-  static_assert(E % 8 == 0, "whole 16-byte groups");
-  constexpr int NW = E / 2;  // packed pairs per thread
+  static_assert(E % 8 == 0 && E <= 64, "whole 16-byte groups, 64-bit masks");
+  static_assert(NT == 128 || NT == 256, "two or one histogram bins per thread");
+  constexpr int NW = E / 2;       // packed pairs per thread
+  constexpr int B1 = 256 / NT;    // pass-1 bins per thread
   __shared__ uint32_t hist[256];
   __shared__ uint32_t sums[8];
   __shared__ float red[8];
@@ -282,7 +325,8 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   auto key_hi = [](uint32_t v) { return (v >> 16) & 0x7FFFu; };
 
   // pass 1: high 8 bits of the key
-  hist[t] = 0u;
+#pragma unroll
+  for (int b = 0; b < B1; ++b) hist[t + NT * b] = 0u;
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < NW; ++j) {
@@ -291,11 +335,18 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   }
   __syncthreads();
   {
-    const uint32_t c = hist[255 - t];
-    const uint32_t s = block_scan_256(c, sums);  // keys in bins >= 255 - t
-    if (s >= static_cast<uint32_t>(k) && s - c < static_cast<uint32_t>(k)) {
-      sel[0] = 255 - t;
-      sel[1] = s - c;
+    // thread t holds bins 255 - B1 t - i, i < B1 (descending)
+    uint32_t cb[B1], c = 0u;
+#pragma unroll
+    for (int i = 0; i < B1; ++i) { cb[i] = hist[255 - B1 * t - i]; c += cb[i]; }
+    uint32_t above = block_scan<NT>(c, sums) - c;  // keys in higher bins
+#pragma unroll
+    for (int i = 0; i < B1; ++i) {
+      if (above < static_cast<uint32_t>(k) && above + cb[i] >= static_cast<uint32_t>(k)) {
+        sel[0] = 255 - B1 * t - i;
+        sel[1] = above;
+      }
+      above += cb[i];
     }
   }
   __syncthreads();
@@ -303,7 +354,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   __syncthreads();
 
   // pass 2: low 7 bits inside bin b1
-  hist[t] = 0u;
+  if (t < 128) hist[t] = 0u;
   __syncthreads();
 #pragma unroll
   for (int j = 0; j < NW; ++j) {
@@ -314,7 +365,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
   __syncthreads();
   {
     const uint32_t c = t < 128 ? hist[127 - t] : 0u;
-    const uint32_t s = block_scan_256(c, sums);
+    const uint32_t s = block_scan<NT>(c, sums);
     const uint32_t need = static_cast<uint32_t>(k) - above1;
     if (t < 128 && s >= need && s - c < need) {
       sel[0] = 127 - t;
@@ -327,7 +378,6 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
 
   // keys above T are kept; keys equal to T are kept in column order until
   // k are kept (the block prefix of their counts ranks this thread's)
-  static_assert(E <= 64, "bit masks of 64 bits");
   uint64_t gt = 0u, eq = 0u;
   uint32_t kmax = 0u;  // the row's largest key: the largest kept one (k >= 1 here)
 #pragma unroll
@@ -338,7 +388,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
     kmax = max(kmax, key);
   }
   const uint32_t n_eq = static_cast<uint32_t>(__popcll(eq));
-  const uint32_t rank = block_scan_256(n_eq, sums) - n_eq;  // equal keys in earlier threads
+  const uint32_t rank = block_scan<NT>(n_eq, sums) - n_eq;  // equal keys in earlier threads
   uint64_t keep = gt;
   if (eq) {  // rare: this thread holds keys equal to T; keep its first ones
     const uint32_t take = rank < need_eq ? min(need_eq - rank, n_eq) : 0u;
@@ -348,10 +398,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
       e &= e - 1u;
     }
   }
-  uint32_t keep_bits[(E + 31) / 32];
-#pragma unroll
-  for (int j = 0; j < (E + 31) / 32; ++j) keep_bits[j] = static_cast<uint32_t>(keep >> (32 * j));
-  const float amax = block_max_256(__uint_as_float(kmax << 16), red);
+  const float amax = block_max<NT>(__uint_as_float(kmax << 16), red);
   const float a = fmaxf(amax, kEps);
   const float inv = __fdiv_rn(127.f, a);
   if (t == 0) xs_out[m] = __fdiv_rn(a, 127.f);
@@ -359,7 +406,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
 #pragma unroll
   for (int c = 0; c < E / 8; ++c) {
     if (c * 8 < nvalid) {
-      const uint32_t kb = keep_bits[(8 * c) >> 5] >> ((8 * c) & 31);  // this group's 8 bits
+      const uint32_t kb = static_cast<uint32_t>(keep >> (8 * c)) & 0xFFu;  // this group's 8 bits
       int q[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -369,7 +416,7 @@ __global__ void __launch_bounds__(kQuantThreads) topk_i8_kernel(
       }
       reinterpret_cast<uint2*>(q_out + m * K + base)[c] =
           make_uint2(pack_s8x4(q[0], q[1], q[2], q[3]), pack_s8x4(q[4], q[5], q[6], q[7]));
-      if (mask_out) mask_out[m * (K >> 3) + (base >> 3) + c] = static_cast<uint8_t>(kb & 0xFFu);
+      if (mask_out) mask_out[m * (K >> 3) + (base >> 3) + c] = static_cast<uint8_t>(kb);
     }
   }
 }
@@ -378,13 +425,14 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                            int8_t* q, float* xs, uint8_t* mask, cudaStream_t s) {
   const int kk = static_cast<int>(k), KK = static_cast<int>(K);
   const unsigned grid = static_cast<unsigned>(M);
-  auto go = [&](auto kern) {
-    return launch_kernel(kern, dim3(grid), dim3(kQuantThreads), 0, s, 0u, x, KK, ldx, kk, q, xs, mask);
+  auto go = [&](auto kern, int threads) {
+    return launch_kernel(kern, dim3(grid), dim3(threads), 0, s, 0u, x, KK, ldx, kk, q, xs, mask);
   };
-  if (K <= 8 * kQuantThreads) return go(topk_i8_kernel<8>);
-  if (K <= 16 * kQuantThreads) return go(topk_i8_kernel<16>);
-  if (K <= 32 * kQuantThreads) return go(topk_i8_kernel<32>);
-  return go(topk_i8_kernel<64>);
+  if (K <= 8 * 128) return go(topk_i8_kernel<128, 8>, 128);
+  if (K <= 16 * 128) return go(topk_i8_kernel<128, 16>, 128);
+  if (K <= 32 * 128) return go(topk_i8_kernel<128, 32>, 128);
+  if (K <= 32 * 256) return go(topk_i8_kernel<256, 32>, 256);
+  return go(topk_i8_kernel<256, 64>, 256);
 }
 
 // ------------------------------------------------------------ KV 3-bit
