@@ -254,6 +254,7 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
   // ring (every load has landed and been unpacked, every MMA has retired)
   __syncthreads();
   int32_t* part = reinterpret_cast<int32_t*>(smem + OFF_W);
+  float* xs_s = reinterpret_cast<float*>(smem + OFF_X);  // row scales, on the drained activation ring
   if (warp >= 4 && warp < 8) {
     tc_fence_after();
     const int q = warp & 3;
@@ -266,24 +267,27 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
       for (int i = 0; i < 32; ++i)
         if (col + i < p.npad) part[(col + i) * BNF + nl] = have_acc ? static_cast<int32_t>(r[i]) : 0;
     }
+    if (nl < p.M) xs_s[nl] = __ldg(p.xs + nl);  // all row scales in one round of loads
   }
   cluster_sync();
-  if (rank == 0 && warp >= 4 && warp < 8) {
+  // the cluster's CTAs share the rows of the final reduction: CTA r sums the
+  // partials of rows r, r + csize, ... over every CTA's shared memory
+  if (warp >= 4 && warp < 8) {
     const int nl = (warp & 3) * 32 + lane;
     const int nn = n0 + nl;
     const float gm = gamma_of(p, nn);
     const uint32_t local = smem_u32(part);
     uint32_t base[8];
     for (int r = 0; r < p.csize; ++r) base[r] = map_shared_rank(local, r);
-    for (int m = 0; m < p.M; ++m) {
+    for (int m = static_cast<int>(rank); m < p.M; m += p.csize) {
       int32_t acc = 0;
       const uint32_t off = 4u * static_cast<uint32_t>(m * BNF + nl);
       for (int r = 0; r < p.csize; ++r) acc += ld_dsmem_s32(base[r] + off);
-      const float f = __fmul_rn(static_cast<float>(acc), __fmul_rn(__ldg(p.xs + m), gm));
+      const float f = __fmul_rn(static_cast<float>(acc), __fmul_rn(xs_s[m], gm));
       p.y[static_cast<int64_t>(m) * p.ldy + nn] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
     }
   }
-  cluster_sync();  // peers keep their shared memory until rank 0 is done
+  cluster_sync();  // every CTA keeps its shared memory until the others are done
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();
