@@ -436,15 +436,17 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 }
 
 // ------------------------------------------------------------ KV 3-bit
-// Each thread quantises 8 consecutive head dims (one 16-byte load); the
-// G = D/8 threads of one (token, head) row reduce their absmax with a
-// segmented warp shuffle. A warp covers 32/G whole rows whose 3-bit
-// streams (3 bytes per thread) form 96 contiguous bytes, staged in shared
-// memory and written as 24 aligned words. The list of 4-bit tokens is copied
-// to shared memory once per block (up to kKeepSmem entries) and searched
-// there; row -> (token, head) uses 32-bit division.
+// Each thread quantises 16 consecutive head dims (two 16-byte loads); the
+// G = D/16 threads of one (token, head) row reduce their absmax with a
+// segmented warp shuffle, so the per-row work (the shuffles, the divisions,
+// the 4-bit list search) is shared by 16 elements a thread. A warp covers
+// 32/G whole rows whose 3-bit streams (6 bytes per thread) form 192
+// contiguous bytes, staged in shared memory and written as 48 aligned words.
+// The list of 4-bit tokens is copied to shared memory once per block (up to
+// kKeepSmem entries) and searched there; row -> (token, head) uses 32-bit
+// division.
 constexpr int kKeepSmem = 1024;
-constexpr int KV_TILES = 4;  // warp tiles per warp (16-byte loads in flight per thread)
+constexpr int KV_TILES = 2;  // warp tiles per warp (2 x 16-byte loads in flight per thread each)
 
 template <int G>
 __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
@@ -452,9 +454,9 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
     int n4, uint8_t* __restrict__ codes3, uint8_t* __restrict__ codes4, float* __restrict__ scale) {
   pdl_wait();  // inputs come from the previous kernel in the stream
   pdl_trigger();
-  constexpr int D = 8 * G;
+  constexpr int D = 16 * G;
   constexpr int RPW = 32 / G;  // rows per warp tile
-  __shared__ __align__(16) uint8_t stage[kQuantThreads / 32][96];
+  __shared__ __align__(16) uint8_t stage[kQuantThreads / 32][192];
   __shared__ int32_t s_keep[kKeepSmem];
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
   const int n4s = n4 < kKeepSmem ? n4 : kKeepSmem;
@@ -462,13 +464,20 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
   const int g = lane % G;
   // this warp's KV_TILES consecutive warp tiles: all loads issued up front
   const uint32_t tile0 = (blockIdx.x * (kQuantThreads / 32) + wid) * KV_TILES;
-  float f[KV_TILES][8];
+  float f[KV_TILES][16];
 #pragma unroll
   for (int j = 0; j < KV_TILES; ++j) {
     const uint32_t row = (tile0 + j) * RPW + lane / G;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) f[j][i] = 0.f;
-    if (row < rows) bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(kv + static_cast<size_t>(row) * D) + g), f[j]);
+    for (int i = 0; i < 16; ++i) f[j][i] = 0.f;
+    if (row < rows) {
+      const uint4* src = reinterpret_cast<const uint4*>(kv + static_cast<size_t>(row) * D) + 2 * g;
+      float lo[8], hi[8];
+      bf16x8_to_f32(__ldg(src), lo);
+      bf16x8_to_f32(__ldg(src + 1), hi);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { f[j][i] = lo[i]; f[j][8 + i] = hi[i]; }
+    }
   }
   __syncthreads();  // s_keep ready
 #pragma unroll
@@ -478,7 +487,7 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
     const bool valid = row < rows;
     float amax = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[j][i]));
+    for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[j][i]));
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
     const uint32_t t = row / H, h = row - t * H;
@@ -496,31 +505,60 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
     const float Q = four ? 7.f : 3.f;
     const float a = fmaxf(amax, kEps);
     const float inv = __fdiv_rn(Q, a);
-    uint32_t packed3 = 0u;
+    uint64_t pk = 0u;  // 48 bits of 3-bit codes
     if (four) {
-      uint32_t packed4 = 0u;
+      uint32_t q0 = 0u, q1 = 0u;
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        packed4 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -8.f, 7.f) + 8) << (4 * i);
+      for (int i = 0; i < 8; ++i) {
+        q0 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -8.f, 7.f) + 8) << (4 * i);
+        q1 |= static_cast<uint32_t>(quant_code(f[j][8 + i], inv, -8.f, 7.f) + 8) << (4 * i);
+      }
       if (valid)
-        reinterpret_cast<uint32_t*>(codes4 + (static_cast<size_t>(jk) * H + h) * (D / 2))[g] = packed4;
+        reinterpret_cast<uint2*>(codes4 + (static_cast<size_t>(jk) * H + h) * (D / 2))[g] = make_uint2(q0, q1);
     } else {
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        packed3 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -4.f, 3.f) + 4) << (3 * i);
+      for (int i = 0; i < 16; ++i)
+        pk |= static_cast<uint64_t>(quant_code(f[j][i], inv, -4.f, 3.f) + 4) << (3 * i);
     }
+    const uint32_t p0 = static_cast<uint32_t>(pk), p1 = static_cast<uint32_t>(pk >> 32);
     if (valid && g == 0) scale[row] = __fdiv_rn(a, Q);
-    stage[wid][3 * lane + 0] = static_cast<uint8_t>(packed3);
-    stage[wid][3 * lane + 1] = static_cast<uint8_t>(packed3 >> 8);
-    stage[wid][3 * lane + 2] = static_cast<uint8_t>(packed3 >> 16);
+    // 6 bytes at offset 6 lane: a 4-byte and a 2-byte store in either order
+    uint8_t* sp = &stage[wid][6 * lane];
+    if ((lane & 1) == 0) {
+      *reinterpret_cast<uint32_t*>(sp) = p0;
+      *reinterpret_cast<uint16_t*>(sp + 4) = static_cast<uint16_t>(p1);
+    } else {
+      *reinterpret_cast<uint16_t*>(sp) = static_cast<uint16_t>(p0);
+      *reinterpret_cast<uint32_t*>(sp + 2) = (p0 >> 16) | (p1 << 16);
+    }
     __syncwarp();
     const int64_t rows_here = static_cast<int64_t>(rows) - warp_row0;
-    const int nbytes = rows_here >= RPW ? 96 : static_cast<int>(rows_here > 0 ? rows_here : 0) * 3 * G;
-    if (lane * 4 < nbytes)
-      reinterpret_cast<uint32_t*>(codes3 + static_cast<size_t>(warp_row0) * (3 * G))[lane] =
-          reinterpret_cast<const uint32_t*>(stage[wid])[lane];
+    const int nbytes = rows_here >= RPW ? 192 : static_cast<int>(rows_here > 0 ? rows_here : 0) * 6 * G;
+    uint32_t* dst = reinterpret_cast<uint32_t*>(codes3 + static_cast<size_t>(warp_row0) * (6 * G));
+    const uint32_t* src = reinterpret_cast<const uint32_t*>(stage[wid]);
+    if (lane * 4 < nbytes) dst[lane] = src[lane];
+    if ((lane + 32) * 4 < nbytes) dst[lane + 32] = src[lane + 32];
     __syncwarp();
   }
+}
+
+cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
+                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
+                            float* scale, cudaStream_t s) {
+  const uint32_t rows = static_cast<uint32_t>(T * H);  // the entry point bounds rows * G < 2^32
+  const int G = static_cast<int>(D / 16);
+  const uint64_t threads = static_cast<uint64_t>(rows) * G;
+  const uint64_t per_block = static_cast<uint64_t>(kQuantThreads) * KV_TILES;
+  const unsigned grid = static_cast<unsigned>((threads + per_block - 1) / per_block);
+  const int n = static_cast<int>(n4);
+  const uint32_t h = static_cast<uint32_t>(H);
+  auto go = [&](auto kern) {
+    return launch_kernel(kern, dim3(grid), dim3(kQuantThreads), 0, s, 0u, kv, rows, h, keep4, n,
+                         codes3, codes4, scale);
+  };
+  if (G == 4) return go(kv_quant_kernel<4>);
+  if (G == 8) return go(kv_quant_kernel<8>);
+  return go(kv_quant_kernel<16>);
 }
 
 // ------------------------------------------------ 4-bit token positions
@@ -574,23 +612,5 @@ cudaError_t launch_keep4_positions(const int32_t* ids, int64_t T, const int32_t*
                        pos, count);
 }
 
-cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
-                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
-                            float* scale, cudaStream_t s) {
-  const uint32_t rows = static_cast<uint32_t>(T * H);  // the entry point bounds rows * G < 2^32
-  const int G = static_cast<int>(D / 8);
-  const uint64_t threads = static_cast<uint64_t>(rows) * G;
-  const uint64_t per_block = static_cast<uint64_t>(kQuantThreads) * KV_TILES;
-  const unsigned grid = static_cast<unsigned>((threads + per_block - 1) / per_block);
-  const int n = static_cast<int>(n4);
-  const uint32_t h = static_cast<uint32_t>(H);
-  auto go = [&](auto kern) {
-    return launch_kernel(kern, dim3(grid), dim3(kQuantThreads), 0, s, 0u, kv, rows, h, keep4, n,
-                         codes3, codes4, scale);
-  };
-  if (G == 8) return go(kv_quant_kernel<8>);
-  if (G == 16) return go(kv_quant_kernel<16>);
-  return go(kv_quant_kernel<32>);
-}
 
 }  // namespace blt
