@@ -88,6 +88,8 @@ __global__ void __launch_bounds__(kQuantThreads) quant_act_kernel(
   const int nchunk = K >> 3;
 
   float amax = 0.f;
+  // unrolled so that several rows' worth of 16-byte loads are in flight per thread
+#pragma unroll 4
   for (int c = threadIdx.x; c < nchunk; c += kQuantThreads) {
     float h[8];
     bf16x8_to_f32(__ldg(xr + c), h);
