@@ -258,19 +258,64 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) { h[i] = a[i]; h[8 + i] = b[i]; }
     };
+    // When every thread has at most two 16-element groups, the raw bf16 words
+    // stay in registers from the first pass to the second (one round of
+    // global loads); otherwise the second pass reads them again.
+    const int ngroups = p.M * G16;
+    const bool held = ngroups <= 2 * static_cast<int>(blockDim.x);
+    uint4 xv[2][2], uv[2][2];
+    if (held) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        xv[r][0] = xv[r][1] = uv[r][0] = uv[r][1] = make_uint4(0u, 0u, 0u, 0u);
+        if (i < ngroups) {
+          const int t = i / G16, g = i - t * G16;
+          const uint4* xr = reinterpret_cast<const uint4*>(p.x + static_cast<int64_t>(t) * p.ldx) + 2 * g;
+          xv[r][0] = __ldg(xr);
+          xv[r][1] = __ldg(xr + 1);
+          if (relu2) {
+            const uint4* ur = reinterpret_cast<const uint4*>(p.up + static_cast<int64_t>(t) * p.ldx) + 2 * g;
+            uv[r][0] = __ldg(ur);
+            uv[r][1] = __ldg(ur + 1);
+          }
+        }
+      }
+    }
+    auto held16 = [&](int r, float (&h)[16]) {
+      float a[8], b[8];
+      act_vals8(xv[r][0], uv[r][0], relu2, a);
+      act_vals8(xv[r][1], uv[r][1], relu2, b);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) { h[i] = a[i]; h[8 + i] = b[i]; }
+    };
     // pass 1: absmax of every token row
     float am[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) am[t] = 0.f;
-    for (int i = threadIdx.x; i < p.M * G16; i += blockDim.x) {
-      const int t = i / G16, g = i - t * G16;
-      float h[16];
-      load16(t, g, h);
+    auto absmax16 = [&](int t, const float (&h)[16]) {
       float mx = 0.f;
 #pragma unroll
       for (int j = 0; j < 16; ++j) mx = fmaxf(mx, fabsf(h[j]));
 #pragma unroll
       for (int u = 0; u < MT; ++u) am[u] = (u == t) ? fmaxf(am[u], mx) : am[u];
+    };
+    if (held) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        if (i < ngroups) {
+          float h[16];
+          held16(r, h);
+          absmax16(i / G16, h);
+        }
+      }
+    } else {
+      for (int i = threadIdx.x; i < ngroups; i += blockDim.x) {
+        float h[16];
+        load16(i / G16, i % G16, h);
+        absmax16(i / G16, h);
+      }
     }
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
@@ -291,10 +336,7 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
     int part[MT];
 #pragma unroll
     for (int t = 0; t < MT; ++t) part[t] = 0;
-    for (int i = threadIdx.x; i < p.M * G16; i += blockDim.x) {
-      const int t = i / G16, g = i - t * G16;
-      float h[16];
-      load16(t, g, h);
+    auto codes16 = [&](int t, int g, const float (&h)[16]) {
       float iv = 0.f;
 #pragma unroll
       for (int u = 0; u < MT; ++u) iv = (u == t) ? inv[u] : iv;
@@ -307,6 +349,23 @@ bitlinear_gemv_dp4a_kernel(const Params p) {
 #pragma unroll
       for (int u = 0; u < MT; ++u) part[u] += (u == t) ? bs : 0;
       *reinterpret_cast<uint4*>(xsm + t * K + 16 * g) = regroup16(v);
+    };
+    if (held) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int i = threadIdx.x + r * blockDim.x;
+        if (i < ngroups) {
+          float h[16];
+          held16(r, h);
+          codes16(i / G16, i % G16, h);
+        }
+      }
+    } else {
+      for (int i = threadIdx.x; i < ngroups; i += blockDim.x) {
+        float h[16];
+        load16(i / G16, i % G16, h);
+        codes16(i / G16, i % G16, h);
+      }
     }
 #pragma unroll
     for (int t = 0; t < MT; ++t) {
