@@ -273,6 +273,69 @@ def test_gemv_matches_gemm(M):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
+def _extreme_weights(K, N):
+    """Columns of all +1, all -1 and all 0 weights, then random ternary ones."""
+    rng = np.random.default_rng(K + N)
+    Wf = rng.normal(0.0, 0.02, size=(K, N)).astype(np.float32)
+    Wf[:, 0::4] = 1.0
+    Wf[:, 1::4] = -1.0
+    Wf[:, 2::4] = 0.0
+    Wt, gamma = O.ternarize(Wf, (N,))
+    return Wt, gamma, torch.from_numpy(O.pack_ternary(Wt)).to(DEV), torch.from_numpy(gamma).to(DEV)
+
+
+@pytest.mark.parametrize("M", [257, 64])
+def test_gemm_max_k_extreme_accumulators(M):
+    """K = 32768, the largest the GEMMs take: codes of -128 (and 127) against
+    columns of all +1 / -1 weights reach |acc| = 2^22, the edge of the exact
+    int32 -> fp32 conversion; raw accumulators bit-exact, bf16 within 2 ulp.
+    M = 257 runs the CTA-pair kernel, M = 64 the single-CTA one."""
+    N, K = 32, 32768
+    xq = np.full((M, K), -128, dtype=np.int8)
+    xq[1::3] = 127
+    xq[2::3] = np.random.default_rng(5).integers(-128, 128, size=xq[2::3].shape)
+    Wt, gamma, Wp, gamma_d = _extreme_weights(K, N)
+    xd = torch.from_numpy(xq).to(DEV)
+    acc = B.gemm_w2a8_acc(xd, Wp)
+    B.check_status()
+    want = O.gemm_acc_int(xq, Wt)
+    assert np.abs(want).max() == 128 * K
+    assert np.array_equal(host(acc).astype(np.int64), want)
+    xs = np.full(M, 1.0 / 127.0, dtype=np.float32)
+    y = B.gemm_w2a8(xd, torch.from_numpy(xs).to(DEV), Wp, gamma_d, (N,))
+    B.check_status()
+    _, y_o = O.bitlinear_int(xq, xs, Wt, gamma, (N,))
+    assert_bf16_close(bits(y), y_o)
+
+
+def test_gemm_fp4_max_k_extreme_accumulators():
+    """FP4 at K = 32768 with every code +-6 (the e2m1 extremes): the fp32
+    accumulators reach 6 K = 196608, still exact."""
+    M, N, K = 257, 32, 32768
+    codes = np.full((M, K), 0x7, dtype=np.uint8)  # +6
+    codes[1::2] = 0xF                              # -6
+    Wt, _, Wp, _ = _extreme_weights(K, N)
+    acc = B.gemm_w2fp4_acc(torch.from_numpy(O.pack_nibbles(codes)).to(DEV), Wp)
+    B.check_status()
+    want = O.gemm_acc_fp4(codes, Wt)
+    assert np.abs(want).max() == 6 * K
+    assert np.array_equal(host(acc).astype(np.float64), want)
+
+
+@pytest.mark.parametrize("M", [1, 64])
+def test_gemv_max_k_extreme_codes(M):
+    """The decode paths at K = 32768 (CUDA-core for one token, tensor-core for
+    64) with codes of -128 against all-+1 / all--1 rows."""
+    N, K = 256, 32768
+    xq = np.full((M, K), -128, dtype=np.int8)
+    xs = np.full(M, 1.0 / 127.0, dtype=np.float32)
+    Wt, gamma, Wp, gamma_d = _extreme_weights(K, N)
+    y = B.gemv_w2(torch.from_numpy(xq).to(DEV), torch.from_numpy(xs).to(DEV), Wp, gamma_d, (N,))
+    B.check_status()
+    _, y_o = O.bitlinear_int(xq, xs, Wt, gamma, (N,))
+    assert_bf16_close(bits(y), y_o)
+
+
 def test_empty_inputs_are_noops():
     e = torch.empty((0, 256), dtype=torch.bfloat16, device=DEV)
     q, xs = B.quant_act(e, O.MODE_INT8)
