@@ -97,6 +97,14 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   using L = Layout<PAIR, MX>;
   constexpr int S_TMA = L::S_TMA, S_W = L::S_W, S_B = L::S_B, BK = L::BK, A_BYTES = L::A_BYTES;
   constexpr int BN = L::BN_T;
+  // FP4 on pairs (a light unpack, so its per-k-block waits and arrivals
+  // weigh): the 8 unpack warps form two groups of UW = 4 that take alternate
+  // k-blocks, one group's waits overlapping the other's work. int8 (an
+  // unpack 3x heavier, the shared-memory port already saturated) keeps all
+  // 8 warps on every k-block, which measured faster.
+  constexpr int UW = MX ? 4 : 8;
+  constexpr uint32_t NUG = 8 / UW;  // unpack groups
+  constexpr int UT = UW * 32;       // unpack threads per k-block
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -122,8 +130,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < S_TMA; ++i) { mbar_init(&afull[i], 1); mbar_init(&empty[i], 1); }
-    for (int i = 0; i < S_W; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], 8); }
-    for (int i = 0; i < S_B; ++i) { mbar_init(&bfull[i], PAIR ? 16 : 8); mbar_init(&bempty[i], 1); }
+    for (int i = 0; i < S_W; ++i) { mbar_init(&wfull[i], 1); mbar_init(&wempty[i], UW); }
+    for (int i = 0; i < S_B; ++i) { mbar_init(&bfull[i], PAIR ? 2 * UW : UW); mbar_init(&bempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], PAIR ? 8 : 4); }
     mbar_init(mma_done, 1);
     *s_abort = 0;
@@ -396,12 +404,14 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     if (lane == 0) bulk_wait_all();  // output stores complete before the CTA exits
   } else if (warp >= 8) {
     // ------------------------------------------------------------- unpack
-    const int ut = threadIdx.x - 256;  // 0..255
+    const uint32_t ugrp = static_cast<uint32_t>(warp - 8) / UW;  // takes k-blocks it % NUG == ugrp
+    const int ut = threadIdx.x - 256 - static_cast<int>(ugrp) * UT;  // 0..UT-1
     const uint32_t bfull_addr0 = lead(&bfull[0]);
     uint32_t it = 0;
     bool ok = true;
     for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride) {
       for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+        if (it % NUG != ugrp) continue;
         const uint32_t s = it % S_W, ph = (it / S_W) & 1;
         const uint32_t b = it % S_B, bph = (it / S_B) & 1;
         if (!mbar_wait(&wfull[s], ph, tmo, s_abort) || !mbar_wait(&bempty[b], bph ^ 1, tmo, s_abort)) {
@@ -416,16 +426,17 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           // the iterations)
           // two packed words (32 k) -> one 16-byte group of 32 e2m1 nibbles
           // (even k low), chunk c of the row's 128-byte swizzled line
-          constexpr int NI = (L::BROWS * 8) / 256;
+          constexpr int NI = (L::BROWS * 8) / UT;
+          static_assert((L::BROWS * 8) % UT == 0, "whole groups per thread");
           uint2 wv[NI];
 #pragma unroll
           for (int i = 0; i < NI; ++i) {
-            const int g = ut + 256 * i;
+            const int g = ut + UT * i;
             wv[i] = ld_shared_v2(src + (g >> 3) * (BK / 4) + 8 * (g & 7));
           }
 #pragma unroll
           for (int i = 0; i < NI; ++i) {
-            const int g = ut + 256 * i;
+            const int g = ut + UT * i;
             const int n = g >> 3, c = g & 7;
             uint4 o;
             e2m1_words(wv[i].x, o.x, o.y);
@@ -435,9 +446,10 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         } else {
           // one word at a time: with the shared-memory port saturated by the
           // MMA and TMA traffic, batching the loads was not faster here
+          static_assert((L::BROWS * WPR) % UT == 0, "whole words per thread");
 #pragma unroll
-          for (int i = 0; i < (L::BROWS * WPR) / 256; ++i) {
-            const int w = ut + 256 * i;          // packed word index in the tile
+          for (int i = 0; i < (L::BROWS * WPR) / UT; ++i) {
+            const int w = ut + UT * i;           // packed word index in the tile
             const int n = w / WPR, j = w % WPR;  // row, 16-deep K group
             const int sub = j >> 3, c = j & 7;   // 128-deep chunk, 16-byte column in it
             const uint32_t word = ld_shared_u32(src + 4 * w);
