@@ -16,21 +16,26 @@
 //
 // Persistent, warp-specialised kernel. In the CTA-pair form (two CTAs of a
 // cluster on one TPC, tcgen05 cta_group::2) a pair owns a 256-token x
-// 256-output tile: each CTA loads its own 128 token rows of activations and
-// unpacks its own 128 weight rows, and one MMA of M = 256 reads both CTAs'
-// shared memory, so each SM stages half of the unpacked weights (the
-// single-CTA form stages all 256 rows and is used for M <= 128).
-//   warp 0      TMA producer: activation tile (128 rows x 128 B, 128-byte
-//               swizzle) and packed-weight tile (128 or 256 rows x 32 B) into
-//               one ring slot
+// 256-output tile (192 for mxf4): each CTA loads its own 128 token rows of
+// activations and unpacks its own half of the weight rows, and one MMA of
+// M = 256 reads both CTAs' shared memory, so each SM stages half of the
+// unpacked weights (the single-CTA form stages all 256 rows and is used for
+// M <= 128). A k-block is 256 deep on pairs, 128 on single CTAs.
+//   warp 0      TMA producer of the activation tiles (one box per k-block,
+//               128-byte swizzle; on pairs the completion goes to the even
+//               CTA's barrier)
+//   warp 2      TMA producer of the packed-weight tiles (K/4 bytes per row)
 //   warp 1      TMEM allocator; in the even CTA the single-thread MMA issuer
-//               (4 MMAs of K = 32 per 128-deep k-block, accumulator in TMEM)
-//   warps 4-7   epilogue: tcgen05.ld (lane = token row), scale, bf16 pack,
-//               16-byte global stores; two TMEM accumulators so the epilogue
-//               of one tile overlaps the mainloop of the next
-//   warps 8-15  unpack: 2-bit weights -> int8 / padded e2m1 K-major tiles in
-//               the swizzled layout the MMA descriptors describe, then
-//               fence.proxy.async and an mbarrier arrive (on the even CTA)
+//               (K = 32 per MMA for kind::i8 / f8f6f4, 64 for mxf4; the
+//               accumulator in TMEM)
+//   warps 4-7   epilogue: tcgen05.ld (lane = token row, 64 columns at a
+//               time), scale, bf16 pack, 128-byte-swizzled staging and one
+//               TMA store per 32 x 64 block; two TMEM accumulators so the
+//               epilogue of one tile overlaps the mainloop of the next
+//   warps 8-15  unpack: 2-bit weights -> int8 / e2m1 K-major tiles in the
+//               swizzled layout the MMA descriptors describe, then
+//               fence.proxy.async and an mbarrier arrive (on the even CTA);
+//               for mxf4 two groups of 4 warps take alternate k-blocks
 // All waits are bounded (see ptx.cuh); a timeout sets a status bit and the
 // CTA unwinds, releasing TMEM.
 #include "common.cuh"
