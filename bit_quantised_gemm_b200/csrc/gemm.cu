@@ -5,12 +5,12 @@
 //                                          for CTA pairs, kind::f8f6f4 else)
 //   y[m, n]   = bf16(acc * (xs[m] * gamma[group(n)]))   (or the raw acc)
 //
-// FP4 on CTA pairs runs at the full 4-bit tensor rate through the
-// block-scaled kind::mxf4: A and B are packed e2m1 (two per byte, 128 bytes =
-// 256 k per swizzled row, half the shared-memory bytes of the padded
-// f8f6f4 form), and every ue8m0 block scale is 1.0 (0x7F), written once into
-// tensor memory at start-up, so the products and their fp32 sums are those
-// of the unscaled codes. The scale columns take part of tensor memory, so
+// FP4 on CTA pairs (K a multiple of 256) runs at the full 4-bit tensor rate
+// through the block-scaled kind::mxf4: A and B are packed e2m1 (two per
+// byte, 128 bytes = 256 k per swizzled row, half the shared-memory bytes of
+// the padded f8f6f4 form that other K take), and every ue8m0 block scale
+// is 1.0 (0x7F), written once into tensor memory at start-up, so the
+// products and their fp32 sums are those of the unscaled codes. The scale columns take part of tensor memory, so
 // these tiles are 192 outputs wide (two accumulators of 192 columns + the
 // scales in 512).
 //
@@ -20,7 +20,8 @@
 // activations and unpacks its own half of the weight rows, and one MMA of
 // M = 256 reads both CTAs' shared memory, so each SM stages half of the
 // unpacked weights (the single-CTA form stages all 256 rows and is used for
-// M <= 128). A k-block is 256 deep on pairs, 128 on single CTAs.
+// M <= 128). A k-block is 256 deep on pairs (512 for mxf4: one 32 KB
+// activation box either way), 128 on single CTAs.
 //   warp 0      TMA producer of the activation tiles (one box per k-block,
 //               128-byte swizzle; on pairs the completion goes to the even
 //               CTA's barrier)
@@ -54,18 +55,21 @@ constexpr int TMEM_COLS = 512;
 // A TMA instruction costs the issuing thread a few hundred ns whatever its
 // size, so the CTA-pair form moves 256-deep k-blocks (32 KB of activations in
 // one 3-D box) and splits the activation and weight loads over two warps.
-// MX: block-scaled FP4 on CTA pairs (packed e2m1 operands, 192-wide tiles).
+// MX: block-scaled FP4 on CTA pairs (packed e2m1 operands, 192-wide tiles);
+// a 512-deep k-block keeps its activation box at 32 KB (two 128-byte
+// swizzled chunks of 256 k), so one instruction per ring slot still suffices
+// at the 4-bit MMA rate.
 template <bool PAIR, bool MX = false>
 struct Layout {
   static constexpr int BN_T = MX ? 192 : BN;        // output columns per tile
-  static constexpr int BK = PAIR ? 256 : 128;       // k-block depth in elements
-  static constexpr int KSUB = BK / 128;             // 128-deep swizzled chunks per k-block (int8)
-  static constexpr int S_TMA = MX ? 6 : PAIR ? 4 : 5;  // activation ring
-  static constexpr int S_W = MX ? 4 : PAIR ? 2 : 4;    // packed-weight ring
+  static constexpr int BK = MX ? 512 : PAIR ? 256 : 128;  // k-block depth in elements
+  static constexpr int KSUB = 2;                    // pair: 128-byte swizzled chunks per k-block
+  static constexpr int S_TMA = MX ? 3 : PAIR ? 4 : 5;  // activation ring
+  static constexpr int S_W = MX ? 3 : PAIR ? 2 : 4;    // packed-weight ring
   static constexpr int S_B = MX ? 3 : PAIR ? 2 : 3;    // unpacked-weight ring
   static constexpr int BROWS = PAIR ? BN_T / 2 : BN_T;  // weight rows staged per CTA
   static constexpr int ROW_BYTES = MX ? BK / 2 : BK;    // bytes of one k-block row in smem
-  static constexpr int A_BYTES = MX ? BM * ROW_BYTES : KSUB * SUB;
+  static constexpr int A_BYTES = BM * ROW_BYTES;
   static constexpr int WP_BYTES = BROWS * (BK / 4);
   static constexpr int B_BYTES = BROWS * ROW_BYTES;
   static constexpr int SF_COL = 2 * BN_T;           // MX: first tensor-memory column of the scales
@@ -78,6 +82,8 @@ struct Layout {
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(!PAIR || A_BYTES == KSUB * SUB, "pair k-block = two 128-byte chunks");
+  static_assert(B_BYTES % 1024 == 0 && (BROWS * 128) % 1024 == 0, "swizzle atoms aligned");
 };
 
 struct Params {
@@ -93,12 +99,12 @@ struct Params {
   uint64_t timeout_ns;
 };
 
-template <bool FP4, bool PAIR>
+template <bool FP4, bool PAIR, bool MX>
 __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                       const __grid_constant__ CUtensorMap tmW,
                       const __grid_constant__ CUtensorMap tmY, const Params p) {
-  constexpr bool MX = FP4 && PAIR;
+  static_assert(!MX || (FP4 && PAIR), "mxf4 is the FP4 CTA-pair form");
   using L = Layout<PAIR, MX>;
   constexpr int S_TMA = L::S_TMA, S_W = L::S_W, S_B = L::S_B, BK = L::BK, A_BYTES = L::A_BYTES;
   constexpr int BN = L::BN_T;
@@ -205,10 +211,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (!mbar_wait(act ? &empty[s] : &wempty[s], ph ^ 1, tmo, s_abort)) { fail(); ok = false; break; }
           if (act) {
             uint8_t* dst = smem + L::OFF_A + s * A_BYTES;
-            if (MX) {  // packed e2m1 rows: one 128-byte (256 k) box column per k-block
-              if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
-              tma_load_2d_pair(dst, &tmA, lead(&afull[s]), kb * (BK / 2), m0);
-            } else if (PAIR) {
+            if (PAIR) {  // two 128-byte swizzled chunks (int8: 128 k each, e2m1: 256 k)
               if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
               tma_load_3d_pair(dst, &tmA, lead(&afull[s]), 0, m0, kb * L::KSUB);
             } else {
@@ -257,12 +260,17 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (!got) { fail(); ok = false; break; }
           tc_fence_after();
           if constexpr (MX) {
-            // 4 MMAs of K = 64 (32 bytes of packed e2m1) along the 128-byte rows
-            const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES);
-            const uint64_t bdesc = smem_desc_sw128(sB + b * L::B_BYTES);
+            // 8 MMAs of K = 64 (32 bytes of packed e2m1), 4 along each 128-byte
+            // chunk; a chunk wholly past K (the second one of the last
+            // k-block when K % 512 = 256) is skipped
 #pragma unroll
-            for (int kk = 0; kk < BK / 64; ++kk)
-              mma_mxf4_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, sfa, sfb, (kb | kk) != 0);
+            for (int kk = 0; kk < BK / 64; ++kk) {
+              const int sub = kk >> 2, k4 = kk & 3;
+              if (sub > 0 && kb * BK + sub * 256 >= p.K) break;
+              const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES + sub * SUB);
+              const uint64_t bdesc = smem_desc_sw128(sB + b * L::B_BYTES + sub * L::BROWS * 128);
+              mma_mxf4_pair(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, sfa, sfb, (kb | kk) != 0);
+            }
           } else
 #pragma unroll
           for (int kk = 0; kk < BK / 32; ++kk) {
@@ -430,23 +438,27 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           // (the ordered shared-memory accesses would otherwise serialise
           // the iterations)
           // two packed words (32 k) -> one 16-byte group of 32 e2m1 nibbles
-          // (even k low), chunk c of the row's 128-byte swizzled line
-          constexpr int NI = (L::BROWS * 8) / UT;
-          static_assert((L::BROWS * 8) % UT == 0, "whole groups per thread");
+          // (even k low): group j of a row goes to 16-byte column j % 8 of
+          // its 128-byte swizzled line in chunk j / 8
+          constexpr int GPR = BK / 32;  // groups per weight row
+          constexpr int NI = (L::BROWS * GPR) / UT;
+          static_assert((L::BROWS * GPR) % UT == 0, "whole groups per thread");
           uint2 wv[NI];
 #pragma unroll
           for (int i = 0; i < NI; ++i) {
             const int g = ut + UT * i;
-            wv[i] = ld_shared_v2(src + (g >> 3) * (BK / 4) + 8 * (g & 7));
+            wv[i] = ld_shared_v2(src + (g / GPR) * (BK / 4) + 8 * (g % GPR));
           }
 #pragma unroll
           for (int i = 0; i < NI; ++i) {
             const int g = ut + UT * i;
-            const int n = g >> 3, c = g & 7;
+            const int n = g / GPR, j = g % GPR;
+            const int sub = j >> 3, c = j & 7;
             uint4 o;
             e2m1_words(wv[i].x, o.x, o.y);
             e2m1_words(wv[i].y, o.z, o.w);
-            st_shared_v4(dst + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4), o.x, o.y, o.z, o.w);
+            st_shared_v4(dst + sub * (L::BROWS * 128) + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4),
+                         o.x, o.y, o.z, o.w);
           }
         } else {
           // one word at a time: with the shared-memory port saturated by the
@@ -517,12 +529,12 @@ static cudaError_t make_map_2d(CUtensorMap* map, CUtensorMapDataType dt, const v
   return cudaSuccess;
 }
 
-template <bool FP4, bool PAIR>
+template <bool FP4, bool PAIR, bool MX = false>
 static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, const CUtensorMap& tmY,
                             const gemm::Params& p, cudaStream_t s) {
   using namespace gemm;
-  using L = Layout<PAIR, FP4 && PAIR>;
-  auto kern = bitlinear_gemm_kernel<FP4, PAIR>;
+  using L = Layout<PAIR, MX>;
+  auto kern = bitlinear_gemm_kernel<FP4, PAIR, MX>;
   static bool attr_set = false;  // once per process (not during graph capture)
   if (!attr_set) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -545,19 +557,24 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   // CTA pairs once there are two 128-row halves to fill; their 3-D activation
   // view needs whole 128-deep K chunks
   const bool pair = a.M > BM && a.K % 128 == 0;
-  const bool mx = pair && fp4;  // block-scaled FP4 on packed operands
+  // block-scaled FP4 on packed operands; its activation view needs whole
+  // 256-deep chunks (other FP4 pairs take kind::f8f6f4 on padded codes)
+  const bool mx = pair && fp4 && a.K % 256 == 0;
   const int bn = mx ? Layout<true, true>::BN_T : BN;
   const int brows = pair ? bn / 2 : bn;
-  const int BK = pair ? Layout<true>::BK : Layout<false>::BK;
+  const int BK = mx ? Layout<true, true>::BK : pair ? Layout<true>::BK : Layout<false>::BK;
   CUtensorMap tmA, tmW, tmY;
   cudaError_t e;
   const CUtensorMapDataType adt = fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   const uint64_t row_bytes = fp4 ? a.K / 2 : a.K;
   if (mx) {
-    // packed e2m1 codes as bytes [M][K/2]: 128 rows x 128 bytes (256 k) per
-    // box, 128-byte swizzle; a ragged last k-block reads zeros past K
-    e = make_map_2d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, a.K / 2, a.M, row_bytes, BK / 2, BM,
-                    CU_TENSOR_MAP_SWIZZLE_128B, why);
+    // packed e2m1 codes as bytes [K/256 chunks][M rows][128 bytes]: one box
+    // = 2 chunks x 128 rows (512 k), two 128-byte-swizzled tiles back to
+    // back; a chunk past K reads zeros
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(a.M), static_cast<cuuint64_t>(a.K / 256)};
+    const cuuint64_t strides[2] = {row_bytes, 128u};
+    const cuuint32_t box[3] = {128, BM, static_cast<cuuint32_t>(Layout<true, true>::KSUB)};
+    e = make_map_3d(&tmA, CU_TENSOR_MAP_DATA_TYPE_UINT8, a.xq, dims, strides, box, why);
   } else if (pair) {
     // [K/128 chunks][M rows][128 elements]: one box = 2 chunks x 128 rows,
     // i.e. two standard 128-byte-swizzled 128 x 128 tiles back to back
@@ -600,6 +617,7 @@ cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char*
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
 
+  if (mx) return launch_t<true, true, true>(tmA, tmW, tmY, p, s);
   if (fp4) return pair ? launch_t<true, true>(tmA, tmW, tmY, p, s) : launch_t<true, false>(tmA, tmW, tmY, p, s);
   return pair ? launch_t<false, true>(tmA, tmW, tmY, p, s) : launch_t<false, false>(tmA, tmW, tmY, p, s);
 }

@@ -168,7 +168,7 @@ def prep_weights(K, N, groups, seed):
 
 GEMM_SHAPES = [  # (M, N, K): single tile, ragged M/N, half k-block, many tiles
     (16, 256, 256), (1, 16, 64), (130, 272, 320), (257, 512, 1024), (2048, 4096, 256),
-    (300, 768, 2048 + 64), (384, 400, 384)]
+    (300, 768, 2048 + 64), (384, 400, 384), (300, 400, 768)]
 
 
 @pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
