@@ -17,7 +17,9 @@ alone over the replicas, timed the same way.
 
 Also reported (same run, rank 0, unless --no-breakdown): the o_proj top-k
 INT8 GEMM, the down_proj ReLU^2 INT8 GEMM, the decode layer at batch 1/8/64
-(weight GB/s) and the 3-bit KV quantiser (GB/s).
+(weight GB/s), the 3-bit KV quantiser (GB/s), the 3-bit KV attention, and
+library references on the prefill shapes (cuBLAS int8 / fp8 / mxfp4 GEMMs on
+plain operands, a read-only HBM stream).
 
 --impl reference times the CPU oracle on host cores on a bounded sample of
 the same workload (rows of X), in the same metric.
@@ -53,6 +55,8 @@ GU = (D, (FFN, 2 * FFN))
 OPS_PER_STEP = 2 * (2 * M_TOK * D * 3 * D + 2 * M_TOK * D * 2 * FFN)
 # nominal dense ratios to bf16 (2.25 PF): int8 4.5 P, fp8 4.5 P, fp4 9 P
 RATIO_INT8, RATIO_FP4 = 2.0, 4.0
+# nominal B200 dense peaks (vendor figures) and ~8 TB/s HBM, reported beside the measured ones
+NOMINAL = {"int8_tops": 4500.0, "fp8_tflops": 4500.0, "fp4_tflops": 9000.0, "hbm_gbs": 8000.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 GEMM_SRC = os.path.join(ROOT, "bit_quantised_gemm_b200", "csrc", "gemm.cu")
 # DRAM bytes per launch of the INT4-path qkv GEMM from one ncu capture, with
@@ -74,7 +78,7 @@ def parse():
                     help="launch without programmatic dependent launch (each kernel waits for "
                          "the previous one before it starts)")
     ap.add_argument("--section", default=None,
-                    help="run only one breakdown section (o_proj, down_proj, decode, kv, kv_attn), e.g. "
+                    help="run only one breakdown section (o_proj, down_proj, decode, kv, kv_attn, library), e.g. "
                          "to profile its kernels; prints that section's JSON")
     return ap.parse_args()
 
@@ -357,8 +361,9 @@ def bench_ours(args, ws, rank, local):
     for n in GEMM_NAMES:
         tops = GEMM_OPS[n] / (kms[n] * 1e-3) / 1e12
         pk = int8_peak if "w2a4" in n else fp4_peak
+        nom = NOMINAL["int8_tops"] if "w2a4" in n else NOMINAL["fp4_tflops"]
         kernels[n] = {"us": round(kms[n] * 1e3, 2), "TOPS": round(tops, 1),
-                      "frac_of_peak": round(tops / pk, 4),
+                      "frac_of_peak": round(tops / pk, 4), "frac_of_nominal": round(tops / nom, 4),
                       "peak": "int8" if "w2a4" in n else "fp4 (tcgen05 kind::mxf4, block scales 1.0)"}
 
     value = OPS_PER_STEP * args.steps * ws / (ms * 1e-3) / 1e12
@@ -518,7 +523,7 @@ def _dev_bf16(torch, bits, dev):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
 
-SECTIONS = ("o_proj", "down_proj", "decode", "kv", "kv_attn")
+SECTIONS = ("o_proj", "down_proj", "decode", "kv", "kv_attn", "library")
 
 
 def breakdown(ctx, args, sections=SECTIONS):
@@ -769,6 +774,78 @@ def section_kv_attn(B, torch, dev, stream, peaks, steps, warm):
         out[f"queries{nq}"] = {"us": round(ms * 1e3, 2), "GBps": round(byt / ms / 1e6, 1),
                                "frac_hbm": round(byt / ms / 1e6 / hbm, 4)}
     return {"kv_attention_3bit_4096x32x128": dict(cache_bytes=cache_bytes, **out)}
+
+
+def section_library(B, torch, dev, stream, peaks, steps, warm):
+    """Library references on the prefill shapes (not this library's kernels):
+    cuBLAS int8 GEMM (torch._int_mm) and fp8 e4m3 GEMM (torch._scaled_mm, unit
+    scales) on plain 8-bit operands with no unpack, an mxfp4 torch._scaled_mm
+    where this torch offers it, and a read-only HBM stream (a torch sum over
+    2 GiB). Each timed like the kernels above over 3 operand replicas."""
+    out = {}
+    int8_peak, hbm = RATIO_INT8 * peaks["bf16_tflops"], peaks["hbm_gbs"]
+    shapes = {"qkv": (M_TOK, D, 3 * D), "gate_up": (M_TOK, D, 2 * FFN)}
+
+    def rate(name, M, K, N, fn_make, peak, nominal):
+        try:
+            calls = [fn_make() for _ in range(3)]
+            ms = time_calls(torch, stream, calls, steps, warm)
+            tops = 2 * M * K * N / (ms * 1e-3) / 1e12
+            out[name] = {"us": round(ms * 1e3, 2), "TOPS": round(tops, 1),
+                         "frac_of_peak": round(tops / peak, 4), "frac_of_nominal": round(tops / nominal, 4)}
+        except Exception as e:  # an unsupported dtype or shape in this torch / cuBLAS
+            out[name] = {"unavailable": f"{type(e).__name__}: {str(e).splitlines()[0][:160]}"}
+        torch.cuda.synchronize()
+
+    for sh, (M, K, N) in shapes.items():
+        def mk_i8(M=M, K=K, N=N):
+            a = torch.randint(-8, 8, (M, K), dtype=torch.int8, device=dev)
+            b = torch.randint(-1, 2, (N, K), dtype=torch.int8, device=dev).t()
+            return lambda: torch._int_mm(a, b)
+        rate(f"cublas_int8_{sh}", M, K, N, mk_i8, int8_peak, NOMINAL["int8_tops"])
+
+        def mk_f8(M=M, K=K, N=N):
+            a = torch.randn(M, K, device=dev).to(torch.float8_e4m3fn)
+            b = torch.randn(N, K, device=dev).to(torch.float8_e4m3fn).t()
+            one = torch.ones((), device=dev)
+            return lambda: torch._scaled_mm(a, b, one, one, out_dtype=torch.bfloat16)
+        rate(f"cublaslt_fp8_{sh}", M, K, N, mk_f8, RATIO_INT8 * peaks["bf16_tflops"], NOMINAL["fp8_tflops"])
+
+        def mk_f4(M=M, K=K, N=N):
+            a = torch.randint(0, 256, (M, K // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2)
+            b = torch.randint(0, 256, (N, K // 2), dtype=torch.uint8, device=dev).view(torch.float4_e2m1fn_x2).t()
+            # every e8m0 block scale 1.0 (127): the same in any scale layout, so
+            # the first layout this torch accepts is used
+            import torch.nn.functional as F
+            err = None
+            for swz in ("SWIZZLE_32_4_4", "NO_SWIZZLE"):
+                for flat in (True, False):
+                    shp_a, shp_b = ((M * K // 32,), (N * K // 32,)) if flat else ((M, K // 32), (N, K // 32))
+                    sa = torch.full(shp_a, 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+                    sb = torch.full(shp_b, 127, dtype=torch.uint8, device=dev).view(torch.float8_e8m0fnu)
+                    bw, sw = F.ScalingType.BlockWise1x32, getattr(F.SwizzleType, swz)
+                    call = (lambda sa=sa, sb=sb, bw=bw, sw=sw: F.scaled_mm(
+                        a, b, sa, bw, sb, bw, swizzle_a=sw, swizzle_b=sw, output_dtype=torch.bfloat16))
+                    try:
+                        call()
+                        return call
+                    except (RuntimeError, ValueError, TypeError) as e:
+                        err = e
+            raise err
+        rate(f"cublaslt_mxfp4_{sh}", M, K, N, mk_f4, RATIO_FP4 * peaks["bf16_tflops"], NOMINAL["fp4_tflops"])
+
+    try:
+        buf = torch.ones(2 << 30 >> 2, dtype=torch.float32, device=dev)  # 2 GiB
+        ms = time_calls(torch, stream, [lambda: buf.sum()], max(8, steps // 8), warm, per_graph=2)
+        gbs = buf.numel() * 4 / (ms * 1e-3) / 1e9
+        out["hbm_read_stream_2GiB"] = {"us": round(ms * 1e3, 1), "GBps": round(gbs, 1),
+                                       "frac_of_measured_copy": round(gbs / hbm, 4),
+                                       "frac_of_nominal": round(gbs / NOMINAL["hbm_gbs"], 4)}
+        del buf
+    except Exception as e:
+        out["hbm_read_stream_2GiB"] = {"unavailable": f"{type(e).__name__}: {str(e)[:160]}"}
+    torch.cuda.empty_cache()
+    return {"library_reference": out}
 
 
 def main():
