@@ -648,6 +648,15 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
     wdev = [{k: (torch.from_numpy(wp).to(dev), torch.from_numpy(gm).to(dev)) for k, (wp, gm) in packed.items()}
             for _ in range(R)]
     names = tuple(shapes)
+    # the six K = 4096 projections as one grouped launch (q|k|v|o|gate|up
+    # concatenated, one scale group each, one shared input: a weight-streaming
+    # measure, not the layer's data flow), plus down: 2 launches for all 7
+    six = ("q", "k", "v", "o", "gate", "up")
+    g_ends = tuple(int(e) for e in np.cumsum([P[n].N for n in six]))
+    g_wp, g_gm = B.ternarize_pack(np.concatenate([P[n].W for n in six], axis=1), g_ends)
+    g_dev = [(torch.from_numpy(g_wp).to(dev), torch.from_numpy(g_gm).to(dev)) for _ in range(R)]
+    g_bytes = D * g_ends[-1] // 4
+    del g_wp
     dec = {}
     for batch in (1, 4, 8, 64):
         x = _dev_bf16(torch, lay["x"][:batch], dev)
@@ -720,6 +729,15 @@ def section_decode(B, torch, dev, stream, peaks, steps, warm):
             "weight_frac_hbm": round(wbytes / gemv_ms / 1e6 / hbm, 4),
             "layer_weight_GBps_incl_quantisers": round(wbytes / (ms / steps) / 1e6, 1),
             "per_projection": per, **fused}
+        if batch in (1, 8):
+            yg = torch.empty((batch, g_ends[-1]), dtype=torch.bfloat16, device=dev)
+            tg = time_calls(torch, stream, [(lambda r=r: B.gemv_w2(q4, xs4, g_dev[r][0], g_dev[r][1], g_ends,
+                                                                  y=yg)) for r in range(R)], steps, warm)
+            tot = tg + k["down"]
+            dec[f"batch{batch}"]["grouped_7_projections"] = {
+                "launches": 2, "us": round(tot * 1e3, 2), "six_k4096_us": round(tg * 1e3, 2),
+                "weight_GBps": round((g_bytes + shapes["down"][0] * shapes["down"][1] // 4) / tot / 1e6, 1),
+                "weight_frac_hbm": round((g_bytes + shapes["down"][0] * shapes["down"][1] // 4) / tot / 1e6 / hbm, 4)}
     out["decode_llama7b_layer"] = dict(weight_bytes=wbytes, launches_per_layer=7,
                                        gemv_launches="qkv (fused, 3 groups), o, gate_up (fused, 2 groups), down",
                                        **dec)
