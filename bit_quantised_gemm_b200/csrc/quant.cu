@@ -445,8 +445,18 @@ cudaError_t launch_topk_i8(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
 // 32/G whole rows whose 3-bit streams (6 bytes per thread) form 192
 // contiguous bytes, staged in shared memory and written as 48 aligned words.
 // The list of 4-bit tokens is copied to shared memory once per block (up to
-// kKeepSmem entries) and searched there; row -> (token, head) uses 32-bit
-// division.
+// kKeepSmem entries) and searched there by row ranges (token p holds rows
+// [p H, p H + H)), so no division by H is needed on the 3-bit path.
+
+// The rounding bias's share of the packed 3-bit words (fields 0..10 of the
+// low word, 11..15 of the high one), modulo 2^32.
+constexpr uint32_t kv3_bias(int first, int last, int base) {
+  uint32_t b = 0u;
+  for (int i = first; i <= last; ++i) b += 0x4B400000u << (3 * i - base);
+  return b;
+}
+constexpr uint32_t kKv3BiasLo = kv3_bias(0, 10, 0);
+constexpr uint32_t kKv3BiasHi = kv3_bias(11, 15, 32);
 constexpr int kKeepSmem = 1024;
 constexpr int KV_TILES = 2;  // warp tiles per warp (2 x 16-byte loads in flight per thread each)
 
@@ -492,15 +502,15 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
     for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fabsf(f[j][i]));
 #pragma unroll
     for (int o = G / 2; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const uint32_t t = row / H, h = row - t * H;
-    int jk = -1;  // index of t among the 4-bit tokens
+    int jk = -1;  // index of this row's token among the 4-bit tokens
     if (valid && n4 > 0) {
+      // token p holds rows [p H, p H + H): compare rows, no division
       int lo = 0, hi = n4 - 1;
       while (lo <= hi) {
         const int mid = (lo + hi) >> 1;
-        const int p = mid < kKeepSmem ? s_keep[mid] : __ldg(keep4 + mid);
-        if (p == static_cast<int>(t)) { jk = mid; break; }
-        if (p < static_cast<int>(t)) lo = mid + 1; else hi = mid - 1;
+        const uint32_t r0 = static_cast<uint32_t>(mid < kKeepSmem ? s_keep[mid] : __ldg(keep4 + mid)) * H;
+        if (row >= r0 && row - r0 < H) { jk = mid; break; }
+        if (r0 < row) lo = mid + 1; else hi = mid - 1;
       }
     }
     const bool four = jk >= 0;
@@ -515,12 +525,25 @@ __global__ void __launch_bounds__(kQuantThreads) kv_quant_kernel(
         q0 |= static_cast<uint32_t>(quant_code(f[j][i], inv, -8.f, 7.f) + 8) << (4 * i);
         q1 |= static_cast<uint32_t>(quant_code(f[j][8 + i], inv, -8.f, 7.f) + 8) << (4 * i);
       }
+      const uint32_t h = row % H;
       if (valid)
         reinterpret_cast<uint2*>(codes4 + (static_cast<size_t>(jk) * H + h) * (D / 2))[g] = make_uint2(q0, q1);
     } else {
+      // code + 4 comes out of the rounding itself: x * inv + (1.5 * 2^23 + 4)
+      // has the bits 0x4B400000 + code + 4. Every |x * inv| <= 3 (1 + 2^-24),
+      // so each code lies in [-3, 3] and needs no clamp. The biased bits,
+      // shifted to their 3-bit fields, are summed modulo 2^32 (the fields do
+      // not overlap) and the bias's share is removed once per word; field 10
+      // straddles the two words.
+      uint32_t lo = 0u, hi = 0u, r10 = 0u;
 #pragma unroll
-      for (int i = 0; i < 16; ++i)
-        pk |= static_cast<uint64_t>(quant_code(f[j][i], inv, -4.f, 3.f) + 4) << (3 * i);
+      for (int i = 0; i < 16; ++i) {
+        const uint32_t r = __float_as_uint(__fadd_rn(__fmul_rn(f[j][i], inv), 12582916.f));
+        if (i <= 10) lo += r << (3 * i);
+        else hi += r << (3 * i - 32);
+        if (i == 10) r10 = r;
+      }
+      pk = (static_cast<uint64_t>(hi - kKv3BiasHi + ((r10 >> 2) & 1u)) << 32) | (lo - kKv3BiasLo);
     }
     const uint32_t p0 = static_cast<uint32_t>(pk), p1 = static_cast<uint32_t>(pk >> 32);
     if (valid && g == 0) scale[row] = __fdiv_rn(a, Q);
