@@ -259,32 +259,74 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
     tc_fence_after();
     const int q = warp & 3;
     const int nl = q * 32 + lane;
-    for (int col = 0; col < p.npad; col += 32) {
-      uint32_t r[32];
-      tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if (col + i < p.npad) part[(col + i) * BNF + nl] = have_acc ? static_cast<int32_t>(r[i]) : 0;
-    }
     if (nl < p.M) xs_s[nl] = __ldg(p.xs + nl);  // all row scales in one round of loads
+    if (p.csize == 1) {
+      // K is not split: each thread's accumulator row is final, so it goes
+      // from tensor memory to y directly (no partials, no DSMEM round trip)
+      named_bar_sync(1, 128);  // the four epilogue warps: row scales staged
+      const int nn = n0 + nl;
+      const float gm = gamma_of(p, nn);
+      uint16_t* yc = p.y + nn;
+      for (int col = 0; col < p.npad && col < p.M; col += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const int m = col + i;
+          if (m < p.M) {
+            const int32_t acc = have_acc ? static_cast<int32_t>(r[i]) : 0;
+            const float f = __fmul_rn(static_cast<float>(acc), __fmul_rn(xs_s[m], gm));
+            yc[static_cast<int64_t>(m) * p.ldy] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+          }
+        }
+      }
+    } else {
+      for (int col = 0; col < p.npad; col += 32) {
+        uint32_t r[32];
+        tmem_ld32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+          if (col + i < p.npad) part[(col + i) * BNF + nl] = have_acc ? static_cast<int32_t>(r[i]) : 0;
+      }
+    }
   }
   cluster_sync();
   // the cluster's CTAs share the rows of the final reduction: CTA r sums the
-  // partials of rows r, r + csize, ... over every CTA's shared memory
-  if (warp >= 4 && warp < 8) {
+  // partials of rows r, r + csize, ... over every CTA's shared memory. Rows
+  // go in groups of 8 so that a thread has 8 DSMEM loads in flight per CTA
+  // rather than one dependent load at a time.
+  if (p.csize > 1 && warp >= 4 && warp < 8) {
     const int nl = (warp & 3) * 32 + lane;
     const int nn = n0 + nl;
     const float gm = gamma_of(p, nn);
     const uint32_t local = smem_u32(part);
     uint32_t base[8];
     for (int r = 0; r < p.csize; ++r) base[r] = map_shared_rank(local, r);
-    for (int m = static_cast<int>(rank); m < p.M; m += p.csize) {
-      int32_t acc = 0;
-      const uint32_t off = 4u * static_cast<uint32_t>(m * BNF + nl);
-      for (int r = 0; r < p.csize; ++r) acc += ld_dsmem_s32(base[r] + off);
-      const float f = __fmul_rn(static_cast<float>(acc), __fmul_rn(xs_s[m], gm));
-      p.y[static_cast<int64_t>(m) * p.ldy + nn] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+    const int step = p.csize;
+    for (int m0 = static_cast<int>(rank); m0 < p.M; m0 += 8 * step) {
+      int32_t acc[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) acc[j] = 0;
+      for (int r = 0; r < p.csize; ++r) {
+        int32_t v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int m = min(m0 + j * step, p.npad - 1);  // rows past M read padding, never stored
+          v[j] = ld_dsmem_s32(base[r] + 4u * static_cast<uint32_t>(m * BNF + nl));
+        }
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[j] += v[j];
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int m = m0 + j * step;
+        if (m < p.M) {
+          const float f = __fmul_rn(static_cast<float>(acc[j]), __fmul_rn(xs_s[m], gm));
+          p.y[static_cast<int64_t>(m) * p.ldy + nn] = __bfloat16_as_ushort(__float2bfloat16_rn(f));
+        }
+      }
     }
   }
   cluster_sync();  // every CTA keeps its shared memory until the others are done
