@@ -49,7 +49,8 @@ constexpr int OFF_X = OFF_W + S_W * W_BYTES;
 constexpr int OFF_BAR = OFF_X + S_X * X_BYTES;
 constexpr int N_BARS = 2 * S_W + 2 * S_X + 2 * RA + 2;
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
-constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+constexpr int OFF_SCALES = OFF_MISC + 16;    // row scales [64], then gamma [8]
+constexpr int SMEM_BYTES = OFF_SCALES + (64 + 8) * 4 + 1024;
 constexpr int THREADS = 384;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(D_COLS + RA * 128 <= TMEM_COLS, "tensor memory budget");
@@ -68,11 +69,12 @@ struct Params {
   uint64_t timeout_ns;
 };
 
-__device__ __forceinline__ float gamma_of(const Params& p, int n) {
+// Scale of output feature n's column group, from the copy in shared memory.
+__device__ __forceinline__ float gamma_of(const Params& p, const float* gam_s, int n) {
   int g = 0;
 #pragma unroll
   for (int i = 0; i < 7; ++i) g += (i < p.G - 1 && n >= p.group_end[i]) ? 1 : 0;
-  return __ldg(p.gamma + g);
+  return gam_s[g];
 }
 
 __device__ __forceinline__ int32_t ld_dsmem_s32(uint32_t addr) {
@@ -116,6 +118,8 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
   uint64_t* mma_done = tfull + 1;
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+  float* xs_s = reinterpret_cast<float*>(smem + OFF_SCALES);  // row scales [M]
+  float* gam_s = xs_s + 64;                                    // group scales [G]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   const uint32_t rank = cluster_ctarank();
@@ -174,10 +178,14 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
     }
   } else if (warp == 2) {
     // ---------------------------------------------- TMA: activation codes
+    // activation codes and row scales come from the previous kernel (y is
+    // written after the block-wide barrier that follows this wait). The
+    // warp stages the row and group scales in shared memory here, so that
+    // the epilogue reads no global memory before its stores.
+    pdl_wait();
+    for (int m = lane; m < p.M; m += 32) xs_s[m] = __ldg(p.xs + m);
+    if (lane < p.G) gam_s[lane] = __ldg(p.gamma + lane);
     if (lane == 0) {
-      // activation codes come from the previous kernel (the row scales and y
-      // are touched after the block-wide barrier that follows this wait)
-      pdl_wait();
       int last = -1;
       for (int c = 0; c < nch; ++c) {
         const uint32_t s = c % S_X, ph = (c / S_X) & 1;
@@ -254,18 +262,15 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
   // ring (every load has landed and been unpacked, every MMA has retired)
   __syncthreads();
   int32_t* part = reinterpret_cast<int32_t*>(smem + OFF_W);
-  float* xs_s = reinterpret_cast<float*>(smem + OFF_X);  // row scales, on the drained activation ring
   if (warp >= 4 && warp < 8) {
     tc_fence_after();
     const int q = warp & 3;
     const int nl = q * 32 + lane;
-    if (nl < p.M) xs_s[nl] = __ldg(p.xs + nl);  // all row scales in one round of loads
     if (p.csize == 1) {
       // K is not split: each thread's accumulator row is final, so it goes
       // from tensor memory to y directly (no partials, no DSMEM round trip)
-      named_bar_sync(1, 128);  // the four epilogue warps: row scales staged
       const int nn = n0 + nl;
-      const float gm = gamma_of(p, nn);
+      const float gm = gamma_of(p, gam_s, nn);
       uint16_t* yc = p.y + nn;
       for (int col = 0; col < p.npad && col < p.M; col += 32) {
         uint32_t r[32];
@@ -300,7 +305,7 @@ bitlinear_gemv_kernel(const __grid_constant__ CUtensorMap tmX,
   if (p.csize > 1 && warp >= 4 && warp < 8) {
     const int nl = (warp & 3) * 32 + lane;
     const int nn = n0 + nl;
-    const float gm = gamma_of(p, nn);
+    const float gm = gamma_of(p, gam_s, nn);
     const uint32_t local = smem_u32(part);
     uint32_t base[8];
     for (int r = 0; r < p.csize; ++r) base[r] = map_shared_rank(local, r);
