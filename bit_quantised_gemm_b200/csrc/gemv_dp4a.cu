@@ -141,7 +141,9 @@ __device__ __forceinline__ int dp4a_us(uint32_t a, uint32_t b, int c) {
 // One packed word against the MT tokens' regrouped activation words.
 // NACC = 4: four masks without a shift, accumulators at scales 1, 4, 16, 64
 // (fewest instructions; used for one or two tokens). NACC = 2: one shift,
-// accumulators at scales 1 and 16 (half the registers).
+// accumulators at scales 1 and 16 (half the registers; four tokens).
+// NACC = 1: three shifts, every field at scale 1 in one accumulator (a
+// quarter of the registers; eight tokens, four rows per item).
 template <int MT, int NACC>
 __device__ __forceinline__ void word_dot(uint32_t w, const uint4 (&xv)[MT], int (&acc)[MT][NACC]) {
   if constexpr (NACC == 4) {
@@ -153,6 +155,16 @@ __device__ __forceinline__ void word_dot(uint32_t w, const uint4 (&xv)[MT], int 
       acc[t][1] = dp4a_us(m1, xv[t].y, acc[t][1]);
       acc[t][2] = dp4a_us(m2, xv[t].z, acc[t][2]);
       acc[t][3] = dp4a_us(m3, xv[t].w, acc[t][3]);
+    }
+  } else if constexpr (NACC == 1) {
+    const uint32_t m0 = w & 0x03030303u, m1 = (w >> 2) & 0x03030303u;
+    const uint32_t m2 = (w >> 4) & 0x03030303u, m3 = (w >> 6) & 0x03030303u;
+#pragma unroll
+    for (int t = 0; t < MT; ++t) {
+      acc[t][0] = dp4a_us(m0, xv[t].x, acc[t][0]);
+      acc[t][0] = dp4a_us(m1, xv[t].y, acc[t][0]);
+      acc[t][0] = dp4a_us(m2, xv[t].z, acc[t][0]);
+      acc[t][0] = dp4a_us(m3, xv[t].w, acc[t][0]);
     }
   } else {
     const uint32_t sh = w >> 2;
@@ -173,7 +185,8 @@ __device__ __forceinline__ void word_dot(uint32_t w, const uint4 (&xv)[MT], int 
 template <int NACC>
 __device__ __forceinline__ int combine(const int (&a)[NACC]) {
   if constexpr (NACC == 4) return a[0] + (a[1] >> 2) + (a[2] >> 4) + (a[3] >> 6);
-  else return a[0] + (a[1] >> 4);
+  else if constexpr (NACC == 2) return a[0] + (a[1] >> 4);
+  else return a[0];
 }
 
 __device__ __forceinline__ float warp_max_f(float v) {
@@ -191,7 +204,7 @@ template <int MT, int RW, bool FUSED, int LW>
 __global__ void __launch_bounds__(LW > 0 ? PAIR_WARPS * 32 : MAX_WARPS * 32, LW > 0 ? 2 : 1)
 bitlinear_gemv_dp4a_kernel(const Params p) {
   static_assert(LW == 0 || (!FUSED && LW % 4 == 0), "register activations: codes given");
-  constexpr int NACC = MT <= 2 ? 4 : 2;
+  constexpr int NACC = MT <= 2 ? 4 : (MT == 4 ? 2 : 1);
   constexpr int U = MT <= 2 ? 4 : (MT == 4 ? 2 : 1);  // words per lane per batch of loads
   constexpr int NV = RW * MT;
   extern __shared__ __align__(16) uint8_t smem[];
@@ -626,7 +639,7 @@ static cudaError_t launch_pick_rows(const gemv_cc::Params& p, cudaStream_t s) {
       return launch_mt<MT, 2, FUSED>(p, s);
     }
   }
-  if constexpr (MT <= 4) {  // eight tokens: 2 rows (registers)
+  {  // items of 4 rows share each load of the activation words over twice the weights
     constexpr int W = gemv_cc::MAX_WARPS;
     if (int64_t(p.N) >= int64_t(4) * W * num_sms() &&
         dp4a_shape(MT, 4, p.K, 2 * W, W, gemv_cc::SMEM_LIMIT).warps == W)

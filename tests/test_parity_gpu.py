@@ -230,7 +230,7 @@ def test_gemv_parity(M, N, K):
     assert_bf16_close(bits(y), y_o)
 
 
-@pytest.mark.parametrize("M,N,K", [(1, 12288, 4096), (4, 22016, 4096)])
+@pytest.mark.parametrize("M,N,K", [(1, 12288, 4096), (4, 22016, 4096), (8, 12288, 4096), (6, 22016, 4096)])
 def test_gemv_decode_full_size(M, N, K):
     """Fused q/k/v and gate/up projections of the decode layer at full size."""
     rng = np.random.default_rng(N + M)
@@ -521,6 +521,25 @@ def test_gemv_quant_fused(M, mode, relu2, N, K):
     q, xs = B.quant_act(xd, mode, up=ud)
     y2 = B.gemv_w2(q, xs, Wp, gamma_d, groups)
     assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+
+
+@pytest.mark.parametrize("M,mode,relu2,N", [(8, O.MODE_INT4, False, 12288), (5, O.MODE_INT8, True, 22016)])
+def test_gemv_quant_fused_wide(M, mode, relu2, N):
+    """Five to eight tokens against the fused q/k/v and gate/up widths: items
+    of four weight rows, one accumulator per token and row."""
+    K = 4096
+    rng = np.random.default_rng(M * 11 + N)
+    x = W.outlier_bf16(rng, M, K)[0]
+    up = W.normal_bf16(rng, (M, K)) if relu2 else None
+    groups = (N // 3, 2 * N // 3, N) if N % 3 == 0 else (N // 2, N)
+    Wt, gamma, Wp, gamma_d = prep_weights(K, N, groups, 19)
+    xd = dev_bf16(x)
+    ud = dev_bf16(up) if relu2 else None
+    y = B.gemv_w2_quant(xd, mode, Wp, gamma_d, groups, up=ud)
+    B.check_status()
+    xq_o, xs_o = O.quant_act(x, mode, up_bits=up)
+    _, y_o = O.bitlinear_int(xq_o, xs_o, Wt, gamma, groups)
+    assert_bf16_close(bits(y), y_o)
 
 
 def test_gemv_quant_fused_strided_rows():
