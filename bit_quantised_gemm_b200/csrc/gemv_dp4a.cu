@@ -17,7 +17,8 @@
 //     t & 0x30303030 -> c of elements 16j + {9, 11, 13, 15}     (x16)
 // leave one code per byte, so dp4a against the activation bytes regrouped in
 // that order gives sum_k c[k] x[k] in two integer accumulators (scales 1 and
-// 16). The layer output is acc = sum_k x[k] W_t[k] = sum_k c[k] x[k] - sum_k
+// 16); with eight tokens each field is shifted down to scale 1 first and one
+// accumulator per token and row takes all four. The layer output is acc = sum_k x[k] W_t[k] = sum_k c[k] x[k] - sum_k
 // x[k], exact in int32, followed by the usual epilogue
 //     y = bf16_rne((float)acc * (xs[m] * gamma[g(n)])).
 //
