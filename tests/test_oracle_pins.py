@@ -197,6 +197,7 @@ def test_topk_golden_ties():
         assert O.topk_keep_mask(xb, k)[0].astype(int).tolist() == [int(v) for v in g[f"mask_k{k}"]]
     q, xs, mask = O.topk_sparsify_i8(xb, 4)
     assert q[0].tolist() == [int(v) for v in g["codes_k4"]]
+    assert O.pack_mask_bits(mask).tolist() == [[int(g["mask_k4_byte"][0], 16)]]
 
 
 @pytest.mark.parametrize("K", [64, 255, 4096])
