@@ -108,6 +108,41 @@ def _require_cuda(*ts):
             raise ValueError("expected a CUDA tensor")
 
 
+# bf16 values, or their 16-bit patterns
+_BF16_LIKE = tuple(d for d in (torch.bfloat16, torch.int16, getattr(torch, "uint16", None)) if d is not None)
+
+
+def _need(t, name: str, dtypes, dim: int | None = None, contiguous: bool = False):
+    """Metadata checks the C ABI cannot make (it sees only pointers and sizes)."""
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected {' or '.join(str(d) for d in dtypes)}")
+    if dim is not None and t.dim() != dim:
+        raise ValueError(f"{name}: {t.dim()}-D, expected {dim}-D")
+    if contiguous and not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _check_gemm_operands(a, code_dtype, xs, Wp, gamma, n_groups: int, K: int, y):
+    """Codes [M x *] contiguous, xs fp32 [>= M], Wp uint8 [N x K/4], gamma fp32
+    [>= G], y (when given) bf16 [M x N] with unit column stride."""
+    _need(a, "activation codes", (code_dtype,), 2, contiguous=True)
+    M = a.shape[0]
+    _need(xs, "xs", (torch.float32,), 1, contiguous=True)
+    if xs.numel() < M:
+        raise ValueError(f"xs: {xs.numel()} scales for {M} rows")
+    _need(Wp, "Wp", (torch.uint8,), 2, contiguous=True)
+    if Wp.shape[1] * 4 != K:
+        raise ValueError(f"Wp: rows of {Wp.shape[1]} bytes, expected K/4 = {K // 4}")
+    _need(gamma, "gamma", (torch.float32,), 1, contiguous=True)
+    if gamma.numel() < n_groups:
+        raise ValueError(f"gamma: {gamma.numel()} scales for {n_groups} column groups")
+    if y is not None:
+        _need(y, "y", _BF16_LIKE, 2)
+        if tuple(y.shape) != (M, Wp.shape[0]) or y.stride(1) != 1:
+            raise ValueError(f"y: shape {tuple(y.shape)} / strides {y.stride()}, expected "
+                             f"({M}, {Wp.shape[0]}) with unit column stride")
+
+
 def _rows(t: torch.Tensor) -> tuple[int, int, int]:
     """(M, K, ld) of a 2-D tensor whose rows are contiguous."""
     if t.dim() != 2 or t.stride(1) != 1:
@@ -155,8 +190,20 @@ def ternarize_pack(W: np.ndarray, group_ends) -> tuple[np.ndarray, np.ndarray]:
 def quant_act(x: torch.Tensor, mode: int, up: torch.Tensor | None = None, out=None, xs=None,
               stream=None):
     """Per-token quantiser (INT8 / INT4 / FP4), optionally of relu(x)^2 * up."""
-    _require_cuda(x, up)
+    _need(x, "x", _BF16_LIKE)
+    if up is not None:
+        _need(up, "up", _BF16_LIKE)
     M, K, ld = _rows(x)
+    if out is not None:
+        fp4 = mode == MODE_FP4
+        _need(out, "out", (torch.uint8,) if fp4 else (torch.int8,), 2, contiguous=True)
+        if tuple(out.shape) != (M, K // 2 if fp4 else K):
+            raise ValueError(f"out: shape {tuple(out.shape)} for {M} rows of {K} values")
+    if xs is not None:
+        _need(xs, "xs", (torch.float32,), 1, contiguous=True)
+        if xs.numel() < M:
+            raise ValueError(f"xs: {xs.numel()} scales for {M} rows")
+    _require_cuda(x, up)
     if up is not None and (up.shape != x.shape or up.stride() != x.stride()):
         raise ValueError("up must match x in shape and strides")
     if out is None:
@@ -172,8 +219,17 @@ def quant_act(x: torch.Tensor, mode: int, up: torch.Tensor | None = None, out=No
 def topk_sparsify_i8(x: torch.Tensor, k: int = 0, mask: bool = False, out=None, xs=None,
                      stream=None):
     """Keep the k (default ceil(K/2)) largest |x| per row, zero the rest, INT8."""
-    _require_cuda(x)
+    _need(x, "x", _BF16_LIKE)
     M, K, ld = _rows(x)
+    if out is not None:
+        _need(out, "out", (torch.int8,), 2, contiguous=True)
+        if tuple(out.shape) != (M, K):
+            raise ValueError(f"out: shape {tuple(out.shape)} for {M} rows of {K} values")
+    if xs is not None:
+        _need(xs, "xs", (torch.float32,), 1, contiguous=True)
+        if xs.numel() < M:
+            raise ValueError(f"xs: {xs.numel()} scales for {M} rows")
+    _require_cuda(x)
     if out is None:
         out = torch.empty((M, K), dtype=torch.int8, device=x.device)
     if xs is None:
@@ -186,10 +242,12 @@ def topk_sparsify_i8(x: torch.Tensor, k: int = 0, mask: bool = False, out=None, 
 
 def _gemm(fn: str, a: torch.Tensor, xs, Wp, gamma, group_ends, K: int, y=None, status=None,
           stream=None):
+    ge = np.ascontiguousarray(group_ends, dtype=np.int64)
+    _check_gemm_operands(a, torch.uint8 if fn.endswith("fp4") else torch.int8, xs, Wp, gamma,
+                         len(ge), K, y)
     _require_cuda(a, xs, Wp, gamma)
     M = a.shape[0]
     N = Wp.shape[0]
-    ge = np.ascontiguousarray(group_ends, dtype=np.int64)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     if status is None:
@@ -223,12 +281,25 @@ def gemv_w2(xq, xs, Wp, gamma, group_ends, y=None, status=None, stream=None):
 def gemv_w2_quant(x, mode, Wp, gamma, group_ends, up=None, y=None, status=None, stream=None):
     """Decode-time BitLinear on bf16 activations (1..8 tokens): the per-token
     INT8 / INT4 quantiser (ReLU^2-gated by `up` when given) runs inside the GEMV."""
-    _require_cuda(x, up, Wp, gamma)
+    _need(x, "x", _BF16_LIKE)
+    if up is not None:
+        _need(up, "up", _BF16_LIKE)
     if x.dim() != 2 or x.stride(1) != 1 or (up is not None and up.stride() != x.stride()):
         raise ValueError("x (and up) must be row-major [M x K] with the same row stride")
     M, K = x.shape
-    N = Wp.shape[0]
     ge = np.ascontiguousarray(group_ends, dtype=np.int64)
+    _need(Wp, "Wp", (torch.uint8,), 2, contiguous=True)
+    if Wp.shape[1] * 4 != K:
+        raise ValueError(f"Wp: rows of {Wp.shape[1]} bytes, expected K/4 = {K // 4}")
+    _need(gamma, "gamma", (torch.float32,), 1, contiguous=True)
+    if gamma.numel() < len(ge):
+        raise ValueError(f"gamma: {gamma.numel()} scales for {len(ge)} column groups")
+    if y is not None:
+        _need(y, "y", _BF16_LIKE, 2)
+        if tuple(y.shape) != (M, Wp.shape[0]) or y.stride(1) != 1:
+            raise ValueError(f"y: shape {tuple(y.shape)}, expected ({M}, {Wp.shape[0]}) with unit column stride")
+    _require_cuda(x, up, Wp, gamma)
+    N = Wp.shape[0]
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     if status is None:

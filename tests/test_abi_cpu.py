@@ -161,3 +161,46 @@ def test_error_raises_python_exception():
         B.set_wait_timeout_ns(-5)
     assert ei.value.code == _lib.ERR_INVALID_ARG
     B.set_wait_timeout_ns(2_000_000_000)
+
+
+def test_binding_rejects_malformed_tensors():
+    """The C ABI sees only pointers and sizes, so the binding checks dtypes,
+    shapes and layouts first (CPU tensors: a well-formed call gets as far as
+    the CUDA-tensor check)."""
+    import torch
+    M, K, N = 4, 256, 128
+    xq = torch.zeros((M, K), dtype=torch.int8)
+    xs = torch.ones(M, dtype=torch.float32)
+    Wp = torch.zeros((N, K // 4), dtype=torch.uint8)
+    g = torch.ones(1, dtype=torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.gemm_w2a8(xq, xs, Wp, g, (N,))
+    with pytest.raises(ValueError, match="activation codes: dtype"):
+        B.gemm_w2a8(xq.to(torch.int32), xs, Wp, g, (N,))
+    with pytest.raises(ValueError, match="activation codes: must be contiguous"):
+        B.gemm_w2a8(torch.zeros((M, 2 * K), dtype=torch.int8)[:, ::2], xs, Wp, g, (N,))
+    with pytest.raises(ValueError, match="activation codes: dtype"):
+        B.gemm_w2fp4(xq, xs, Wp, g, (N,))  # FP4 codes are packed uint8
+    with pytest.raises(ValueError, match="xs: dtype"):
+        B.gemv_w2(xq, xs.double(), Wp, g, (N,))
+    with pytest.raises(ValueError, match="xs: 3 scales"):
+        B.gemm_w2a8(xq, xs[:3], Wp, g, (N,))
+    with pytest.raises(ValueError, match="Wp: rows of"):
+        B.gemm_w2a8(xq, xs, Wp[:, :32].contiguous(), g, (N,))
+    with pytest.raises(ValueError, match="gamma: 1 scales for 2"):
+        B.gemm_w2a8(xq, xs, Wp, g, (64, N))
+    with pytest.raises(ValueError, match="y: shape"):
+        B.gemm_w2a8(xq, xs, Wp, g, (N,), y=torch.empty((M, N + 1), dtype=torch.bfloat16))
+    x = torch.zeros((M, K), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.quant_act(x, _lib.MODE_INT4)
+    with pytest.raises(ValueError, match="x: dtype"):
+        B.quant_act(x.float(), _lib.MODE_INT4)
+    with pytest.raises(ValueError, match="out: shape"):
+        B.quant_act(x, _lib.MODE_FP4, out=torch.empty((M, K), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="out: dtype"):
+        B.topk_sparsify_i8(x, out=torch.empty((M, K), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="CUDA"):
+        B.gemv_w2_quant(x, _lib.MODE_INT4, Wp, g, (N,))
+    with pytest.raises(ValueError, match="Wp: dtype"):
+        B.gemv_w2_quant(x, _lib.MODE_INT4, Wp.to(torch.int8), g, (N,))
