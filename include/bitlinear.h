@@ -21,6 +21,8 @@
  *     described as W [K x N] (in x out) and stored transposed and packed.
  *   - M == 0 is a valid empty call: nothing is launched.
  *   - Device pointers to TMA-read operands must be 16-byte aligned.
+ *   - One GPU per process: each kernel's shared-memory attribute is raised
+ *     once, on the device that is current at its first call.
  *   - dev_status (nullable, device int): a kernel that gives up a bounded
  *     wait ORs BITLINEAR_STATUS_TIMEOUT into it and returns early; the
  *     output is then undefined. The caller zeroes it; read it with
