@@ -310,8 +310,17 @@ def gemv_w2_quant(x, mode, Wp, gamma, group_ends, up=None, y=None, status=None, 
     return y
 
 
+def _check_acc_operands(a, code_dtype, Wp, K: int):
+    """Codes [M x *] contiguous, Wp uint8 [N x K/4] contiguous."""
+    _need(a, "activation codes", (code_dtype,), 2, contiguous=True)
+    _need(Wp, "Wp", (torch.uint8,), 2, contiguous=True)
+    if Wp.shape[1] * 4 != K:
+        raise ValueError(f"Wp: rows of {Wp.shape[1]} bytes, expected K/4 = {K // 4}")
+
+
 def gemm_w2a8_acc(xq, Wp, status=None, stream=None):
     """Raw int32 accumulators [M x N] of the int8 GEMM."""
+    _check_acc_operands(xq, torch.int8, Wp, xq.shape[1])
     _require_cuda(xq, Wp)
     M, K = xq.shape
     N = Wp.shape[0]
@@ -324,6 +333,7 @@ def gemm_w2a8_acc(xq, Wp, status=None, stream=None):
 
 def gemm_w2fp4_acc(xf4, Wp, status=None, stream=None):
     """Raw fp32 accumulators [M x N] of the FP4 GEMM."""
+    _check_acc_operands(xf4, torch.uint8, Wp, 2 * xf4.shape[1])
     _require_cuda(xf4, Wp)
     M, Kh = xf4.shape
     N = Wp.shape[0]
@@ -334,20 +344,40 @@ def gemm_w2fp4_acc(xf4, Wp, status=None, stream=None):
     return acc
 
 
+def _check_kv_store(prefix: str, codes3, codes4, scale, T: int, H: int, D: int, n4: int):
+    """The (codes3, codes4, scale) of a 3-bit cache of T tokens, H heads, head
+    dim D with n4 tokens at 4 bits: uint8 [T x H x 3D/8], uint8 [n4 x H x D/2]
+    (None when n4 == 0), fp32 [T x H], all contiguous."""
+    for t, name, dt, shape in ((codes3, "codes3", torch.uint8, (T, H, 3 * D // 8)),
+                               (scale, "scale", torch.float32, (T, H)),
+                               (codes4, "codes4", torch.uint8, (n4, H, D // 2))):
+        if t is None:
+            if name == "codes4" and n4 == 0:
+                continue
+            raise ValueError(f"{prefix}{name}: missing")
+        _need(t, prefix + name, (dt,), len(shape), contiguous=True)
+        if tuple(t.shape) != shape:
+            raise ValueError(f"{prefix}{name}: shape {tuple(t.shape)}, expected {shape}")
+
+
 def kv_quant_3bit(kv: torch.Tensor, keep4_pos: torch.Tensor | None, codes3=None, codes4=None,
                   scale=None, stream=None):
     """3-bit per-(token, head) KV quantiser; listed tokens at 4 bits."""
-    _require_cuda(kv, keep4_pos)
     if kv.dim() != 3 or not kv.is_contiguous():
         raise ValueError("kv must be a contiguous [T x H x D] tensor")
+    _need(kv, "kv", _BF16_LIKE)
     T, H, D = kv.shape
     n4 = 0 if keep4_pos is None else keep4_pos.numel()
+    if keep4_pos is not None:
+        _need(keep4_pos, "keep4_pos", (torch.int32,), 1, contiguous=True)
     if codes3 is None:
         codes3 = torch.empty((T, H, 3 * D // 8), dtype=torch.uint8, device=kv.device)
     if codes4 is None and n4:
         codes4 = torch.empty((n4, H, D // 2), dtype=torch.uint8, device=kv.device)
     if scale is None:
         scale = torch.empty((T, H), dtype=torch.float32, device=kv.device)
+    _check_kv_store("", codes3, codes4, scale, T, H, D, n4)
+    _require_cuda(kv, keep4_pos, codes3, codes4, scale)
     _check(lib().kv_quant_3bit(_ptr(kv), T, H, D, _ptr(keep4_pos), n4, _ptr(codes3), _ptr(codes4),
                                _ptr(scale), _stream(stream)))
     return codes3, codes4, scale
@@ -375,12 +405,23 @@ def kv_attention_3bit(q: torch.Tensor, k_store, v_store, keep4_pos: torch.Tensor
     and v_store are the (codes3, codes4, scale) triples of kv_quant_3bit."""
     k3, k4, ks = k_store
     v3, v4, vs = v_store
-    _require_cuda(q, k3, ks, v3, vs, keep4_pos)
     if q.dim() != 3 or not q.is_contiguous():
         raise ValueError("q must be a contiguous [B x H x D] tensor")
+    _need(q, "q", _BF16_LIKE)
     B, H, D = q.shape
+    if k3.dim() != 3:
+        raise ValueError("k codes3 must be [T x H x 3D/8]")
     T = k3.shape[0]
     n4 = 0 if keep4_pos is None else keep4_pos.numel()
+    if keep4_pos is not None:
+        _need(keep4_pos, "keep4_pos", (torch.int32,), 1, contiguous=True)
+    _check_kv_store("k ", k3, k4, ks, T, H, D, n4)
+    _check_kv_store("v ", v3, v4, vs, T, H, D, n4)
+    if out is not None:
+        _need(out, "out", _BF16_LIKE, 3, contiguous=True)
+        if tuple(out.shape) != (B, H, D):
+            raise ValueError(f"out: shape {tuple(out.shape)}, expected {(B, H, D)}")
+    _require_cuda(q, k3, k4, ks, v3, v4, vs, keep4_pos, out)
     if out is None:
         out = torch.empty((B, H, D), dtype=torch.bfloat16, device=q.device)
     if status is None:

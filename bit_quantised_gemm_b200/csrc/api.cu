@@ -5,7 +5,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <map>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "common.cuh"
@@ -15,7 +17,7 @@
 namespace {
 
 thread_local char g_err[512] = "";
-int64_t g_timeout_ns = 2000000000LL;
+std::atomic<int64_t> g_timeout_ns{2000000000LL};
 std::atomic<bool> g_overlap{false};
 
 int fail(int code, const char* fmt, ...) {
@@ -73,7 +75,7 @@ int check_gemm(const char* fn, const void* xq, const void* xs, const uint8_t* Wp
   a->M = M;
   a->N = N;
   a->K = K;
-  a->timeout_ns = static_cast<uint64_t>(g_timeout_ns);
+  a->timeout_ns = static_cast<uint64_t>(g_timeout_ns.load(std::memory_order_relaxed));
   return BITLINEAR_OK;
 }
 
@@ -120,6 +122,23 @@ int num_sms() {
 
 bool launch_overlap() { return g_overlap.load(std::memory_order_relaxed); }
 
+cudaError_t set_smem_limit(const void* kern, int bytes, bool max_carveout) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  static std::mutex mu;
+  static std::map<std::pair<int, const void*>, int> raised;  // (device, kernel) -> limit set
+  std::lock_guard<std::mutex> lock(mu);
+  int& have = raised[std::make_pair(dev, kern)];
+  if (bytes <= have) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && max_carveout)
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  if (e == cudaSuccess) have = bytes;
+  return e;
+}
+
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s) {
   wait_probe_kernel<<<1, 32, 0, s>>>(status, timeout_ns);
   return cudaGetLastError();
@@ -140,7 +159,7 @@ int bitlinear_set_launch_overlap(int enable) {
 
 int bitlinear_set_wait_timeout_ns(int64_t ns) {
   if (ns <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "timeout must be positive");
-  g_timeout_ns = ns;
+  g_timeout_ns.store(ns, std::memory_order_relaxed);
   return ok();
 }
 
@@ -378,7 +397,7 @@ int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_
   const char* why = nullptr;
   cudaError_t e = blt::launch_kv_attention(q, B, H, D, T, k_codes3, k_codes4, k_scale, v_codes3,
                                            v_codes4, v_scale, keep4_pos, n_keep4, out, dev_status,
-                                           static_cast<uint64_t>(g_timeout_ns), stream, &why);
+                                           static_cast<uint64_t>(g_timeout_ns.load(std::memory_order_relaxed)), stream, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_attention_3bit", why);
 }
 

@@ -369,14 +369,9 @@ kv_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 template <int D, int BG>
 static cudaError_t launch_attn_t(const CUtensorMap (&maps)[4], const attn::Params& p, int S,
                                  cudaStream_t s) {
-  static bool attr_set = false;  // once per process (not during graph capture)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(attn::kv_attention_kernel<D, BG>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(sizeof(attn::Smem<D, BG>)));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit(attn::kv_attention_kernel<D, BG>,
+                                  static_cast<int>(sizeof(attn::Smem<D, BG>)));
+  if (e != cudaSuccess) return e;
   const dim3 grid(static_cast<unsigned>(S), static_cast<unsigned>(p.H),
                   static_cast<unsigned>((p.B + BG - 1) / BG));
   return launch_kernel(attn::kv_attention_kernel<D, BG>, grid, dim3(attn::TT),

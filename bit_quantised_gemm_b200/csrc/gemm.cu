@@ -535,13 +535,8 @@ static cudaError_t launch_t(const CUtensorMap& tmA, const CUtensorMap& tmW, cons
   using namespace gemm;
   using L = Layout<PAIR, MX>;
   auto kern = bitlinear_gemm_kernel<FP4, PAIR, MX>;
-  static bool attr_set = false;  // once per process (not during graph capture)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         L::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit(kern, L::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   const int sms = num_sms();
   if (PAIR) {
     const int pairs = p.num_tiles < sms / 2 ? p.num_tiles : sms / 2;

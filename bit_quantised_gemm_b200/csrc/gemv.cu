@@ -398,13 +398,8 @@ cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why) {
       return cudaErrorInvalidValue;
     }
   }
-  static bool attr_set = false;  // once per process (not during graph capture)
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(bitlinear_gemv_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  cudaError_t e = set_smem_limit(bitlinear_gemv_kernel, SMEM_BYTES);
+  if (e != cudaSuccess) return e;
   return launch_kernel(bitlinear_gemv_kernel, dim3(static_cast<unsigned>(tiles * c)), dim3(THREADS),
                        SMEM_BYTES, s, static_cast<unsigned>(c), tmX, tmW, p);
 }

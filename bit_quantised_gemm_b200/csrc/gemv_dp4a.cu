@@ -617,13 +617,9 @@ static cudaError_t launch_mt(gemv_cc::Params p, cudaStream_t s) {
   p.sw = sh.sw;
   auto kern = regs ? gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED, kRegs ? 8 : 0>
                    : gemv_cc::bitlinear_gemv_dp4a_kernel<MT, RW, FUSED, 0>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(sh.smem));
-  // all of the unified L1 as shared memory, so that a second CTA finds room
-  // without the SM changing its split
-  if (e == cudaSuccess && regs)
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
+  // with register activations, all of the unified L1 as shared memory, so
+  // that a second CTA finds room without the SM changing its split
+  cudaError_t e = set_smem_limit(kern, static_cast<int>(sh.smem), regs);
   if (e != cudaSuccess) return e;
   return launch_kernel(kern, dim3(grid), dim3(sh.warps * 32), sh.smem, s, 0u, p);
 }

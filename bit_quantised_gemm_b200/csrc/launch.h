@@ -65,6 +65,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
 EncodeTiledFn get_encode_tiled();
 int num_sms();
 
+// Raise a kernel's dynamic shared-memory limit on the current device to at
+// least `bytes` (and, with max_carveout, ask for all of the unified L1 as
+// shared memory). Function attributes belong to a device's context, so this
+// is kept per (device, kernel); it is thread-safe, and calls that need no
+// larger limit only take a lock and a lookup.
+cudaError_t set_smem_limit(const void* kern, int bytes, bool max_carveout = false);
+template <typename... A>
+inline cudaError_t set_smem_limit(void (*kern)(A...), int bytes, bool max_carveout = false) {
+  return set_smem_limit(reinterpret_cast<const void*>(kern), bytes, max_carveout);
+}
+
 // Process-wide switch (bitlinear_set_launch_overlap): launch with
 // programmatic stream serialisation so a kernel may start while the previous
 // one in the stream finishes. Every kernel calls pdl_wait() before it reads

@@ -222,12 +222,9 @@ static cudaError_t launch_quant_t(const uint16_t* x, const uint16_t* up, int64_t
     return launch_quant_warp<MODE, RELU2, 16>(x, up, M, K, ldx, q, xs, s);
   const size_t smem = static_cast<size_t>(K) * sizeof(float);
   auto kern = quant_act_kernel<MODE, RELU2>;
-  static int attr_bytes = 48 * 1024;  // raised once, monotonically (outside graph capture in practice)
-  if (static_cast<int>(smem) > attr_bytes) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  if (smem > 48 * 1024) {
+    cudaError_t e = set_smem_limit(kern, static_cast<int>(smem));
     if (e != cudaSuccess) return e;
-    attr_bytes = static_cast<int>(smem);
   }
   return launch_kernel(kern, dim3(static_cast<unsigned>(M)), dim3(kQuantThreads), smem, s, 0u,
                        x, up, K, ldx, q, xs);

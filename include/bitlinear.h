@@ -21,8 +21,9 @@
  *     described as W [K x N] (in x out) and stored transposed and packed.
  *   - M == 0 is a valid empty call: nothing is launched.
  *   - Device pointers to TMA-read operands must be 16-byte aligned.
- *   - One GPU per process: each kernel's shared-memory attribute is raised
- *     once, on the device that is current at its first call.
+ *   - Launches go to the device current on the calling thread. Each kernel's
+ *     shared-memory limit is raised once per device (thread-safe), so one
+ *     process may drive several GPUs.
  *   - dev_status (nullable, device int): a kernel that gives up a bounded
  *     wait ORs BITLINEAR_STATUS_TIMEOUT into it and returns early; the
  *     output is then undefined. The caller zeroes it; read it with
@@ -226,7 +227,8 @@ int kv_keep4_positions(const int32_t* token_ids, int64_t T, const int32_t* speci
  *   out[b,h] = bf16_rne(sum_t p_t v[t,h])
  * with k, v dequantised from the kv_quant_3bit storage ((code) * scale), in
  * fp32 with an online softmax. Agrees with the fp64 result within one bf16
- * ulp plus 2.5e-4 of the largest |v| (fp32 accumulation over T terms).
+ * ulp plus 2^-16 (sum_t p_t |v_t| + |out|) per element (fp32 rounding of
+ * the D-term scores and of the weighted sums).
  *   q          device bf16 [B x H x D]
  *   k_*, v_*   codes3 / codes4 / scale of K and V as written by kv_quant_3bit
  *              with the same keep4_pos list (codes4 nullable iff n_keep4 == 0)

@@ -396,6 +396,19 @@ def kv_dequant(codes3, codes4, scale, keep4_pos, D):
     return out
 
 
+def kv_attention_probs_f64(q_bits, k_store, keep4_pos):
+    """The softmax weights of the decode attention below (reading C10), fp64:
+    p[b, h, t] = softmax_t((q[b,h] . k_t) / sqrt(D)) over every cached token
+    t of head h, k_t the dequantised cache row. Returns p [B x H x T]."""
+    q = bf16_to_f32(q_bits).astype(np.float64)
+    D = q.shape[2]
+    k = kv_dequant(*k_store, keep4_pos, D)  # [T x H x D]
+    s = np.einsum("bhd,thd->bht", q, k) / math.sqrt(D)
+    s = s - s.max(axis=2, keepdims=True)
+    p = np.exp(s)
+    return p / p.sum(axis=2, keepdims=True)
+
+
 def kv_attention_f64(q_bits, k_store, v_store, keep4_pos):
     """Decode attention over the C9 cache (the consumer of the 3-bit KV
     quantiser; [R] "Эксперименты": 3-bit KV cache). The pages state only the
@@ -407,14 +420,9 @@ def kv_attention_f64(q_bits, k_store, v_store, keep4_pos):
 
     q_bits: bf16 bits [B x H x D]; k_store, v_store: (codes3, codes4, scale)
     as returned by kv_quant_3bit. Returns o as fp64 [B x H x D]."""
-    q = bf16_to_f32(q_bits).astype(np.float64)
-    D = q.shape[2]
-    k = kv_dequant(*k_store, keep4_pos, D)  # [T x H x D]
+    D = np.asarray(q_bits).shape[2]
+    p = kv_attention_probs_f64(q_bits, k_store, keep4_pos)
     v = kv_dequant(*v_store, keep4_pos, D)
-    s = np.einsum("bhd,thd->bht", q, k) / math.sqrt(D)
-    s = s - s.max(axis=2, keepdims=True)
-    p = np.exp(s)
-    p = p / p.sum(axis=2, keepdims=True)
     return np.einsum("bht,thd->bhd", p, v)
 
 

@@ -204,3 +204,62 @@ def test_binding_rejects_malformed_tensors():
         B.gemv_w2_quant(x, _lib.MODE_INT4, Wp, g, (N,))
     with pytest.raises(ValueError, match="Wp: dtype"):
         B.gemv_w2_quant(x, _lib.MODE_INT4, Wp.to(torch.int8), g, (N,))
+
+
+def test_binding_rejects_malformed_acc_and_kv_tensors():
+    """The raw-accumulator GEMMs and the KV calls check every operand against
+    the sizes they pass to the C ABI before any launch (a short Wp or v3
+    would otherwise send a tensor map past the end of an allocation)."""
+    import torch
+    M, K, N = 4, 256, 128
+    xq = torch.zeros((M, K), dtype=torch.int8)
+    Wp = torch.zeros((N, K // 4), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.gemm_w2a8_acc(xq, Wp)
+    with pytest.raises(ValueError, match="Wp: rows of"):
+        B.gemm_w2a8_acc(xq, Wp[:, :32].contiguous())
+    with pytest.raises(ValueError, match="activation codes: dtype"):
+        B.gemm_w2a8_acc(xq.to(torch.int16), Wp)
+    with pytest.raises(ValueError, match="Wp: dtype"):
+        B.gemm_w2a8_acc(xq, Wp.to(torch.int8))
+    f4 = torch.zeros((M, K // 2), dtype=torch.uint8)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.gemm_w2fp4_acc(f4, Wp)
+    with pytest.raises(ValueError, match="Wp: rows of"):
+        B.gemm_w2fp4_acc(f4[:, :64].contiguous(), Wp)
+    with pytest.raises(ValueError, match="must be contiguous"):
+        B.gemm_w2fp4_acc(torch.zeros((M, K), dtype=torch.uint8)[:, ::2], Wp)
+
+    T, H, D = 40, 4, 128
+    kv = torch.zeros((T, H, D), dtype=torch.bfloat16)
+    keep = torch.tensor([0], dtype=torch.int32)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.kv_quant_3bit(kv, keep)
+    with pytest.raises(ValueError, match="codes3: shape"):
+        B.kv_quant_3bit(kv, keep, codes3=torch.empty((T, H, D // 4), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="codes4: shape"):
+        B.kv_quant_3bit(kv, keep, codes4=torch.empty((2, H, D // 2), dtype=torch.uint8))
+    with pytest.raises(ValueError, match="scale: dtype"):
+        B.kv_quant_3bit(kv, keep, scale=torch.empty((T, H), dtype=torch.float64))
+    with pytest.raises(ValueError, match="keep4_pos: dtype"):
+        B.kv_quant_3bit(kv, keep.long())
+    with pytest.raises(ValueError, match="kv: dtype"):
+        B.kv_quant_3bit(kv.float(), keep)
+
+    q = torch.zeros((2, H, D), dtype=torch.bfloat16)
+    c3 = torch.zeros((T, H, 3 * D // 8), dtype=torch.uint8)
+    c4 = torch.zeros((1, H, D // 2), dtype=torch.uint8)
+    sc = torch.ones((T, H), dtype=torch.float32)
+    good = (c3, c4, sc)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.kv_attention_3bit(q, good, good, keep)
+    with pytest.raises(ValueError, match="v codes3: shape"):
+        B.kv_attention_3bit(q, good, (c3[:T - 1].contiguous(), c4, sc), keep)
+    with pytest.raises(ValueError, match="v scale: shape"):
+        B.kv_attention_3bit(q, good, (c3, c4, sc[:, :2].contiguous()), keep)
+    with pytest.raises(ValueError, match="k codes4: missing"):
+        B.kv_attention_3bit(q, (c3, None, sc), good, keep)
+    with pytest.raises(ValueError, match="k codes3: shape"):
+        B.kv_attention_3bit(torch.zeros((2, H, 256), dtype=torch.bfloat16), good, good, keep)
+    with pytest.raises(ValueError, match="out: shape"):
+        B.kv_attention_3bit(q, good, good, keep, out=torch.empty((1, H, D), dtype=torch.bfloat16))

@@ -47,6 +47,47 @@ def _nearest_bf16_bruteforce(v: float) -> int:
     return (best[1] >> 16) & 0xFFFF
 
 
+def test_bf16_ulp_diff_hand_pairs():
+    """The checker behind every bf16 parity verdict, on pairs whose distance
+    follows from the bf16 format (1 sign, 8 exponent, 7 mantissa bits)."""
+    pairs = [
+        (0x3F80, 0x3F81, 1),       # 1.0 and the next value up: one mantissa step
+        (0x3F80, 0x3F7F, 1),       # 1.0 and the value below it (exponent changes)
+        (0x0001, 0x8001, 2),       # +/- smallest subnormal: -d -> 0 -> +d
+        (0x0000, 0x8000, 0),       # +0 and -0 are the same value
+        (0x8000, 0x0001, 1),       # -0 (= 0) to the smallest subnormal
+        (0x7F7F, 0x7F7E, 1),       # largest finite and the one below it
+        (0xFF7F, 0xFF7E, 1),       # the same pair, negative
+        (0x3F80, 0x4000, 128),     # 1.0 -> 2.0: the 2^7 mantissa steps of one binade
+        (0xBF80, 0x3F80, 2 * 0x3F80),  # -1 -> +1: every step from 0 to 1, twice
+        (0xC2F6, 0xC2F6, 0),       # equal patterns
+    ]
+    a = np.array([p[0] for p in pairs], np.uint16)
+    b = np.array([p[1] for p in pairs], np.uint16)
+    assert O.bf16_ulp_diff(a, b).tolist() == [p[2] for p in pairs]
+    assert O.bf16_ulp_diff(b, a).tolist() == [p[2] for p in pairs]  # symmetric
+
+
+def test_bf16_ulp_diff_matches_rank_of_finite_values():
+    """Brute force: the distance equals the difference of the two values'
+    ranks among all distinct finite bf16 values in increasing order (+0 and
+    -0 one value), computed from the decoded floats alone."""
+    allbits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    vals = O.bf16_to_f32(allbits)
+    finite = np.isfinite(vals)
+    ranks_of = np.unique(vals[finite])  # sorted distinct values, -0 == +0
+    rng = np.random.default_rng(7)
+    fb = allbits[finite]
+    a = rng.choice(fb, 20000)
+    b = np.where(rng.random(20000) < 0.5, rng.choice(fb, 20000),
+                 (a.astype(np.int32) + rng.integers(-3, 4, 20000)).astype(np.uint16))
+    ok = np.isfinite(O.bf16_to_f32(b))
+    a, b = a[ok], b[ok]
+    ra = np.searchsorted(ranks_of, O.bf16_to_f32(a))
+    rb = np.searchsorted(ranks_of, O.bf16_to_f32(b))
+    assert np.array_equal(O.bf16_ulp_diff(a, b), np.abs(ra - rb))
+
+
 def test_f64_to_bf16_exact_rounding():
     rng = np.random.default_rng(1)
     vals = list(rng.standard_normal(300) * 10.0 ** rng.integers(-5, 5, 300))
