@@ -58,10 +58,10 @@ RATIO_INT8, RATIO_FP4 = 2.0, 4.0
 # nominal B200 dense peaks (vendor figures) and ~8 TB/s HBM, reported beside the measured ones
 NOMINAL = {"int8_tops": 4500.0, "fp8_tflops": 4500.0, "fp4_tflops": 9000.0, "hbm_gbs": 8000.0}
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-GEMM_SRC = os.path.join(ROOT, "bit_quantised_gemm_b200", "csrc", "gemm.cu")
-# DRAM bytes per launch of the INT4-path qkv GEMM from one ncu capture, with
-# the sha256 of the kernel source it was taken on (null once it changes).
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_w2a4_qkv_prefill_2048x2048x6144.md")
+CSRC = os.path.join(ROOT, "bit_quantised_gemm_b200", "csrc")
+# DRAM bytes per launch of a kernel from one ncu capture, with the sha256 of
+# the kernel source it was taken on (the figure reads as null once it changes).
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 
 
 def parse():
@@ -92,21 +92,19 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def read_traffic():
-    """(bytes per launch, source) from the committed ncu summary, or (None, why)."""
+def read_traffic(kernel: str):
+    """(DRAM bytes per launch, source) of `kernel` from profiles/traffic.json,
+    or (None, why) when there is no capture or the source changed since."""
     if not os.path.exists(TRAFFIC_FILE):
         return None, "no ncu capture committed"
-    text = open(TRAFFIC_FILE).read()
-    src_hash = hashlib.sha256(open(GEMM_SRC, "rb").read()).hexdigest()
-    vals = {}
-    for line in text.splitlines():
-        if line.startswith("traffic_bytes_per_launch:"):
-            vals["t"] = float(line.split(":", 1)[1])
-        if line.startswith("kernel_source_sha256:"):
-            vals["h"] = line.split(":", 1)[1].strip()
-    if "t" not in vals or vals.get("h") != src_hash:
+    with open(TRAFFIC_FILE) as f:
+        rec = json.load(f).get(kernel)
+    if rec is None:
+        return None, "no ncu capture of this kernel"
+    src = os.path.join(CSRC, rec["source"])
+    if hashlib.sha256(open(src, "rb").read()).hexdigest() != rec["source_sha256"]:
         return None, "kernel changed since the ncu capture"
-    return vals["t"], "ncu"
+    return float(rec["dram_bytes_per_launch"]), "ncu"
 
 
 # ----------------------------------------------------------------- clocks
@@ -241,11 +239,19 @@ def run_step(B, r: PrefillReplica, ev=None):
 
 LAUNCHES_PER_STEP = 6
 GEMM_NAMES = ("w2a4_qkv", "w2a4_gu", "w2fp4_qkv", "w2fp4_gu")
+GEMM_DESC = {"w2a4_qkv": "gemm_w2a4 q|k|v, tcgen05 kind::i8", "w2a4_gu": "gemm_w2a4 gate|up, tcgen05 kind::i8",
+             "w2fp4_qkv": "gemm_w2fp4 q|k|v, tcgen05 kind::mxf4", "w2fp4_gu": "gemm_w2fp4 gate|up, tcgen05 kind::mxf4"}
+# names in profiles/traffic.json
+KERNEL_IDS = {n: f"gemm_{n}_prefill_2048x2048x{3 * D if 'qkv' in n else 2 * FFN}" for n in
+              ("w2a4_qkv", "w2a4_gu", "w2fp4_qkv", "w2fp4_gu")}
+# algorithmic bytes of one launch: codes (1 B or 1/2 B per element) + packed weights + bf16 output
+GEMM_BYTES = {n: M_TOK * D // (2 if "fp4" in n else 1) + (3 * D if "qkv" in n else 2 * FFN) * D // 4
+              + 2 * M_TOK * (3 * D if "qkv" in n else 2 * FFN) for n in ("w2a4_qkv", "w2a4_gu", "w2fp4_qkv", "w2fp4_gu")}
 GEMM_OPS = {"w2a4_qkv": 2 * M_TOK * D * 3 * D, "w2a4_gu": 2 * M_TOK * D * 2 * FFN,
             "w2fp4_qkv": 2 * M_TOK * D * 3 * D, "w2fp4_gu": 2 * M_TOK * D * 2 * FFN}
 
 
-def make_prefill(B, torch, dev, seed, with_oracle_inputs=False):
+def make_prefill(B, torch, dev, seed):
     import workloads as W
     d = W.input_projection_prefill(seed=seed)
     qkv_p, gu_p = d["projs"]
@@ -320,6 +326,16 @@ def time_calls(torch, stream, calls, steps, warm, per_graph=8):
     return ms / steps / per_graph
 
 
+def measure_tensor_peaks(B, torch, stream, reps=3):
+    """Dense tensor-pipe rates (TOPS) of this GPU in the GEMMs' MMA shapes,
+    best of `reps` (bitlinear_tensor_peak; each run ~2 ms of MMAs)."""
+    out = {}
+    for kind, name, iters in ((0, "i8_pair", 8192), (1, "mxf4_pair", 8192), (2, "i8_cta", 8192)):
+        out[name] = max(B.tensor_peak(kind, iters, stream=stream)["tops"] for _ in range(reps))
+    torch.cuda.synchronize()
+    return out
+
+
 def bench_ours(args, ws, rank, local):
     import torch
     import bit_quantised_gemm_b200 as B
@@ -348,23 +364,37 @@ def bench_ours(args, ws, rank, local):
     peaks, peak_src = load_peaks()
     int8_peak = RATIO_INT8 * peaks["bf16_tflops"]
     fp4_peak = RATIO_FP4 * peaks["bf16_tflops"]
-    ach = GEMM_OPS["w2a4_qkv"] / (kms["w2a4_qkv"] * 1e-3) / 1e12
-    traffic, tsrc = read_traffic()
-    roofline = {"bound": "tensor", "kernel": "gemm_w2a4 qkv (tcgen05 kind::i8)",
-                "achieved": round(ach, 1), "peak": round(int8_peak, 1), "unit": "TOPS",
-                "frac": round(ach / int8_peak, 4), "traffic": traffic, "traffic_source": tsrc,
-                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TF/s x {RATIO_INT8} "
-                               "(nominal int8/bf16 dense ratio)",
+    pipe = measure_tensor_peaks(B, torch, stream)
+    # the roofline is reported on the kernel that takes the largest share of the step
+    dom = max(GEMM_NAMES, key=lambda n: kms[n])
+    dom_int8 = "w2a4" in dom
+    ach = GEMM_OPS[dom] / (kms[dom] * 1e-3) / 1e12
+    traffic, tsrc = read_traffic(KERNEL_IDS[dom])
+    dom_peak = int8_peak if dom_int8 else fp4_peak
+    dom_pipe = pipe["i8_pair"] if dom_int8 else pipe["mxf4_pair"]
+    roofline = {"bound": "tensor", "kernel": f"{dom} ({GEMM_DESC[dom]})",
+                "achieved": round(ach, 1), "peak": round(dom_peak, 1), "unit": "TOPS",
+                "frac": round(ach / dom_peak, 4), "traffic": traffic, "traffic_source": tsrc,
+                "algorithmic_bytes": GEMM_BYTES[dom],
+                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TF/s x "
+                               f"{RATIO_INT8 if dom_int8 else RATIO_FP4} (nominal dense ratio to bf16)",
+                "measured_pipe_peak": round(dom_pipe, 1),
+                "frac_of_measured_pipe": round(ach / dom_pipe, 4),
+                "pipe_peak_source": "bitlinear_tensor_peak in this run: back-to-back tcgen05 MMAs of the "
+                                    "GEMM's own kind and shape on resident operands, every SM",
                 "timing": "the GEMM alone: CUDA graphs of 8 back-to-back launches over the 3 replicas, "
                           "CUDA events on the launching stream"}
     kernels = {}
     for n in GEMM_NAMES:
         tops = GEMM_OPS[n] / (kms[n] * 1e-3) / 1e12
-        pk = int8_peak if "w2a4" in n else fp4_peak
-        nom = NOMINAL["int8_tops"] if "w2a4" in n else NOMINAL["fp4_tflops"]
+        i8 = "w2a4" in n
+        pk = int8_peak if i8 else fp4_peak
+        pp = pipe["i8_pair"] if i8 else pipe["mxf4_pair"]
+        nom = NOMINAL["int8_tops"] if i8 else NOMINAL["fp4_tflops"]
         kernels[n] = {"us": round(kms[n] * 1e3, 2), "TOPS": round(tops, 1),
-                      "frac_of_peak": round(tops / pk, 4), "frac_of_nominal": round(tops / nom, 4),
-                      "peak": "int8" if "w2a4" in n else "fp4 (tcgen05 kind::mxf4, block scales 1.0)"}
+                      "frac_of_peak": round(tops / pk, 4), "frac_of_measured_pipe": round(tops / pp, 4),
+                      "frac_of_nominal": round(tops / nom, 4),
+                      "peak": "int8 (bf16 x 2)" if i8 else "fp4 (bf16 x 4; tcgen05 kind::mxf4, block scales 1.0)"}
 
     value = OPS_PER_STEP * args.steps * ws / (ms * 1e-3) / 1e12
     out = {"metric": METRIC, "value": round(value, 2), "unit": "TOPS", "n_gpus": ws,
@@ -377,7 +407,8 @@ def bench_ours(args, ws, rank, local):
                       "l2": f"{R} rotating replicas of all inputs/weights/outputs (>270 MB > 126 MB L2)",
                       "graphs": "one CUDA graph per step",
                       "launch_overlap": not args.no_overlap},
-           "roofline": roofline, "kernels": kernels, "clocks": clk,
+           "roofline": roofline, "tensor_pipe_peaks_TOPS": {k: round(v, 1) for k, v in pipe.items()},
+           "kernels": kernels, "clocks": clk,
            "gpu_launches": LAUNCHES_PER_STEP * args.steps}
     return out, (d, qkv, gu, reps, B, torch, dev, stream)
 
@@ -473,8 +504,7 @@ def blas_threads():
     return os.cpu_count()
 
 
-def cpu_baseline(d, budget_s=12.0, block=64):
-    qkv_wt, gu_wt = oracle_weights(d)
+def _oracle_rate(d, qkv_wt, gu_wt, budget_s, block):
     ops, t, rows_done = 0.0, 0.0, 0
     while t < budget_s and rows_done < M_TOK:
         rows = np.arange(rows_done, min(M_TOK, rows_done + block))
@@ -482,9 +512,24 @@ def cpu_baseline(d, budget_s=12.0, block=64):
         ops += oracle_sample(d, qkv_wt, gu_wt, rows)
         t += time.perf_counter() - t0
         rows_done += len(rows)
-    return {"value": round(ops / t / 1e12, 6), "unit": "TOPS", "cores": blas_threads(), "kind": "oracle",
-            "sample": f"first {rows_done} of {M_TOK} token rows through both variants "
-                      f"({t:.1f} s of CPU time; weight ternarisation untimed)"}
+    return ops / t / 1e12, rows_done, t
+
+
+def cpu_baseline(d, budget_s=8.0, block=32):
+    """The oracle as it stands on the host cores, on the first token rows of
+    the workload that fit the time budget: once with NumPy's BLAS on every
+    core, once on one thread. A baseline, not a target."""
+    from threadpoolctl import threadpool_limits
+    qkv_wt, gu_wt = oracle_weights(d)
+    v_all, rows_all, t_all = _oracle_rate(d, qkv_wt, gu_wt, budget_s, block)
+    cores = blas_threads()
+    with threadpool_limits(limits=1):
+        v_one, rows_one, t_one = _oracle_rate(d, qkv_wt, gu_wt, budget_s, block)
+    return {"value": round(v_all, 6), "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"first {rows_all} of {M_TOK} token rows through both variants ({t_all:.1f} s of CPU "
+                      f"time; weight ternarisation untimed)",
+            "single_thread": {"value": round(v_one, 6), "unit": "TOPS", "cores": 1,
+                              "sample": f"first {rows_one} token rows ({t_one:.1f} s)"}}
 
 
 def bench_reference(args, ws, rank):
@@ -526,12 +571,14 @@ def _dev_bf16(torch, bits, dev):
 SECTIONS = ("o_proj", "down_proj", "decode", "kv", "kv_attn", "library")
 
 
-def breakdown(ctx, args, sections=SECTIONS):
+def breakdown(ctx, args, sections=SECTIONS, pipe=None):
     """The other workloads of the path, each timed the same way (rotating
     replicas larger than L2, CUDA graphs without event nodes; a kernel's time
-    is that of a graph of back-to-back launches of it alone)."""
+    is that of a graph of back-to-back launches of it alone). `pipe`: the
+    tensor-pipe rates measured in this run (measured here when None)."""
     B, torch, dev, stream = ctx[4], ctx[5], ctx[6], ctx[7]
     peaks, src = load_peaks()
+    peaks = dict(peaks, pipe=pipe if pipe is not None else measure_tensor_peaks(B, torch, stream))
     out = {"peaks": f"{src}: HBM {peaks['hbm_gbs']} GB/s, int8 {RATIO_INT8 * peaks['bf16_tflops']:.0f} "
                     "TOPS (2 x bf16 burst)"}
     steps, warm = max(24, min(args.steps, 200)), min(5, args.warmup)
@@ -573,6 +620,7 @@ def section_o_proj(B, torch, dev, stream, peaks, steps, warm):
         "step_us": round(ms / steps * 1e3, 2),
         "gemm_us": round(k["gemm"] * 1e3, 2), "gemm_TOPS": round(ops / k["gemm"] / 1e9, 1),
         "gemm_frac_int8": round(ops / k["gemm"] / 1e9 / int8_peak, 4),
+        "gemm_frac_of_pipe": round(ops / k["gemm"] / 1e9 / peaks["pipe"]["i8_pair"], 4),
         "topk_us": round(k["topk"] * 1e3, 2), "topk_GBps": round(tb / k["topk"] / 1e6, 1),
         "topk_frac_hbm": round(tb / k["topk"] / 1e6 / hbm, 4)}
     return out
@@ -616,6 +664,7 @@ def section_down_proj(B, torch, dev, stream, peaks, steps, warm):
         "step_us": round(ms / steps * 1e3, 2),
         "gemm_us": round(k["gemm"] * 1e3, 2), "gemm_TOPS": round(ops / k["gemm"] / 1e9, 1),
         "gemm_frac_int8": round(ops / k["gemm"] / 1e9 / int8_peak, 4),
+        "gemm_frac_of_pipe": round(ops / k["gemm"] / 1e9 / peaks["pipe"]["i8_pair"], 4),
         "relu2_quant_us": round(k["quant"] * 1e3, 2), "relu2_quant_GBps": round(qb / k["quant"] / 1e6, 1),
         "relu2_quant_frac_hbm": round(qb / k["quant"] / 1e6 / hbm, 4),
         "zero_code_fraction": round(zero_codes, 4)}
@@ -866,6 +915,41 @@ def section_library(B, torch, dev, stream, peaks, steps, warm):
     return {"library_reference": out}
 
 
+def summary(out):
+    """The headline fractions in a few hundred bytes: GEMMs against the tensor
+    pipe measured in this run, decode GEMVs and the HBM-bound kernels against
+    the measured copy bandwidth."""
+    r = lambda v: round(v, 3) if isinstance(v, float) else v
+    sm = {"prefill_TOPS": out["value"], "roofline_frac": out["roofline"]["frac"],
+          "pipe_TOPS": out.get("tensor_pipe_peaks_TOPS"),
+          "gemm_frac_of_pipe": {n: r(k["frac_of_measured_pipe"]) for n, k in out["kernels"].items()}}
+    b = out.get("breakdown", {})
+    o = b.get("o_proj_topk_w2a8_4096x4096x4096", {})
+    dn = b.get("down_proj_relu2_w2a8_4096x11008x4096", {})
+    if o:
+        sm["gemm_frac_of_pipe"]["o_proj"] = r(o.get("gemm_frac_of_pipe"))
+        sm["topk_frac_hbm"] = r(o.get("topk_frac_hbm"))
+    if dn:
+        sm["gemm_frac_of_pipe"]["down_proj"] = r(dn.get("gemm_frac_of_pipe"))
+        sm["relu2_quant_frac_hbm"] = r(dn.get("relu2_quant_frac_hbm"))
+    dec = b.get("decode_llama7b_layer", {})
+    if dec:
+        sm["decode_weight_frac_hbm"] = {k: r(v["weight_frac_hbm"]) for k, v in dec.items() if k.startswith("batch")}
+        sm["decode_gemv_us"] = {k: r(v["gemv_sum_us"]) for k, v in dec.items() if k.startswith("batch")}
+    kv = b.get("kv_quant_3bit_2x4096x32x128")
+    if kv:
+        sm["kv_quant_frac_hbm"] = r(kv["frac_hbm"])
+    at = b.get("kv_attention_3bit_4096x32x128")
+    if at:
+        sm["kv_attn_frac_hbm"] = {q: r(at[q]["frac_hbm"]) for q in ("queries1", "queries8") if q in at}
+    if "e2e" in out:
+        sm["e2e_TOPS"] = out["e2e"]["value"]
+    if "cpu_baseline" in out:
+        sm["cpu_TOPS"] = {"all_cores": out["cpu_baseline"]["value"],
+                          "one_core": out["cpu_baseline"]["single_thread"]["value"]}
+    return sm
+
+
 def main():
     args = parse()
     ws, rank, local = dist_init()
@@ -888,10 +972,12 @@ def main():
     if not args.no_e2e:
         out["e2e"] = bench_e2e(args, ctx, ws)
     if rank == 0 and ws == 1 and not args.no_breakdown:
-        out["breakdown"] = breakdown(ctx, args)
+        pipe = {k: v for k, v in out["tensor_pipe_peaks_TOPS"].items()}
+        out["breakdown"] = breakdown(ctx, args, pipe=pipe)
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(ctx[0])
     if rank == 0:
+        out["summary"] = summary(out)  # last: the end of the line is what a log tail keeps
         print(json.dumps(out), flush=True)
     if ws > 1:
         import torch.distributed as dist

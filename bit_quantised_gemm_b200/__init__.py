@@ -7,5 +7,5 @@ from ._lib import (  # noqa: F401
     gemm_w2a4, gemm_w2a8, gemm_w2a8_acc, gemm_w2fp4, gemm_w2fp4_acc, gemv_w2, gemv_w2_quant,
     header_functions,
     kv_attention_3bit, kv_keep4_positions, kv_quant_3bit, lib, quant_act, set_launch_overlap, set_wait_timeout_ns, status_buffer, ternarize_pack,
-    topk_sparsify_i8, version,
+    tensor_peak, topk_sparsify_i8, version,
 )

@@ -55,6 +55,7 @@ _SIGS = {
     "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
     "kv_keep4_positions": ([_P, _I64, _P, _INT, _P, _P, _P], _INT),
     "bitlinear_check_status": ([_P, _P], _INT),
+    "bitlinear_tensor_peak": ([_INT, _INT, _P, _P, _P, _P], _INT),
     "bitlinear_debug_wait_timeout": ([_P, _I64, _P], _INT),
 }
 
@@ -429,6 +430,23 @@ def kv_attention_3bit(q: torch.Tensor, k_store, v_store, keep4_pos: torch.Tensor
     _check(lib().kv_attention_3bit(_ptr(q), B, H, D, T, _ptr(k3), _ptr(k4), _ptr(ks), _ptr(v3), _ptr(v4),
                                    _ptr(vs), _ptr(keep4_pos), n4, _ptr(out), _ptr(status), _stream(stream)))
     return out
+
+
+def tensor_peak(kind: int, iters: int = 4096, status=None, stream=None) -> dict:
+    """Dense tensor-pipe rate in the GEMMs' MMA shapes (bitlinear_tensor_peak):
+    kind 0 = kind::i8 CTA pairs 256x256x32, 1 = kind::mxf4 pairs 256x256x64,
+    2 = kind::i8 one CTA 128x256x32. Returns {'tops', 'units', 'max_ns'}."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ns = torch.zeros(torch.cuda.get_device_properties(dev).multi_processor_count, dtype=torch.int64, device=dev)
+    units = _c.c_int(0)
+    status = status if status is not None else status_buffer(dev)
+    _check(lib().bitlinear_tensor_peak(int(kind), int(iters), _ptr(ns), _c.addressof(units), _ptr(status),
+                                       _stream(stream)))
+    (stream or torch.cuda.current_stream()).synchronize()
+    n = units.value
+    max_ns = int(ns[:n].max().item())
+    M, N, K = {0: (256, 256, 32), 1: (256, 256, 64), 2: (128, 256, 32)}[int(kind)]
+    return {"tops": n * 4 * iters * 2 * M * N * K / max_ns * 1e-3, "units": n, "max_ns": max_ns}
 
 
 def check_status(status: torch.Tensor | None = None, stream=None):

@@ -17,7 +17,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libbitlinear.so")
-SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemv.cu", "gemv_dp4a.cu", "attn.cu"]
+SOURCES = ["api.cu", "quant.cu", "gemm.cu", "gemv.cu", "gemv_mma.cu", "gemv_dp4a.cu", "attn.cu", "peak.cu"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

@@ -150,7 +150,7 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 104; }
+int bitlinear_version(void) { return 105; }
 
 int bitlinear_set_launch_overlap(int enable) {
   g_overlap.store(enable != 0);
@@ -310,11 +310,17 @@ int bitlinear_gemv_w2(const int8_t* xq, const float* xs, const uint8_t* Wp, cons
   a.ldo = ldy;
   a.out_mode = blt::kOutBf16;
   a.status = dev_status;
-  if (blt::gemv_dp4a_supported(M, K)) {
+  const char* why = nullptr;
+  // one token: CUDA-core dp4a on the packed codes; 2..8: warp-level MMAs;
+  // more: the tcgen05 GEMV (measured crossovers on the decode layer shapes)
+  if (M == 1 && blt::gemv_dp4a_supported(M, K)) {
     cudaError_t e = blt::launch_gemv_dp4a(a, stream);
     return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2 (dp4a)");
   }
-  const char* why = nullptr;
+  if (blt::gemv_mma_supported(M, N, K)) {
+    cudaError_t e = blt::launch_gemv_mma(a, stream, &why);
+    return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2 (warp MMA)", why);
+  }
   cudaError_t e = blt::launch_gemv(a, stream, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2", why);
 }
@@ -399,6 +405,20 @@ int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_
                                            v_codes4, v_scale, keep4_pos, n_keep4, out, dev_status,
                                            static_cast<uint64_t>(g_timeout_ns.load(std::memory_order_relaxed)), stream, &why);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_attention_3bit", why);
+}
+
+int bitlinear_tensor_peak(int kind, int iters, uint64_t* ns_out, int* units_out, int* dev_status,
+                          bitlinear_stream_t stream) {
+  if (kind < 0 || kind > 2) return fail(BITLINEAR_ERR_INVALID_ARG, "tensor_peak: kind must be 0, 1 or 2");
+  if (iters < 1 || iters > (1 << 22)) return fail(BITLINEAR_ERR_INVALID_ARG, "tensor_peak: iters in 1..2^22");
+  if (!ns_out || !units_out) return fail(BITLINEAR_ERR_INVALID_ARG, "tensor_peak: null pointer");
+  int units = 0;
+  cudaError_t e = blt::launch_tensor_peak(kind, iters, reinterpret_cast<unsigned long long*>(ns_out), dev_status,
+                                          static_cast<uint64_t>(g_timeout_ns.load(std::memory_order_relaxed)),
+                                          &units, stream);
+  if (e != cudaSuccess) return cuda_fail(e, "tensor_peak launch");
+  *units_out = units;
+  return ok();
 }
 
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream) {

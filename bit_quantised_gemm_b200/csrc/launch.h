@@ -46,8 +46,13 @@ struct GemmArgs {
 // encoder is unavailable (message in *why).
 cudaError_t launch_gemm(const GemmArgs& a, bool fp4, cudaStream_t s, const char** why);
 cudaError_t launch_gemv(const GemmArgs& a, cudaStream_t s, const char** why);
-// CUDA-core decode path for few tokens (dp4a on packed codes); larger
-// batches take the tensor-core GEMV.
+// Decode path for up to 8 tokens: warp-level MMAs (mma.sync u8 x s8) on the
+// masked 2-bit codes, weights streamed by TMA before the dependency wait.
+constexpr int kGemvMmaMaxTokens = 8;
+bool gemv_mma_supported(int64_t M, int64_t N, int64_t K);
+cudaError_t launch_gemv_mma(const GemmArgs& a, cudaStream_t s, const char** why);
+// CUDA-core decode path with the activation quantiser inside (dp4a on the
+// packed codes), up to 8 tokens.
 constexpr int kGemvDp4aMaxTokens = 8;
 bool gemv_dp4a_supported(int64_t M, int64_t K);
 cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s);
@@ -56,6 +61,10 @@ cudaError_t launch_gemv_dp4a(const GemmArgs& a, cudaStream_t s);
 cudaError_t launch_gemv_dp4a_quant(const GemmArgs& a, const uint16_t* x, const uint16_t* up,
                                    int64_t ldx, int mode, cudaStream_t s);
 cudaError_t launch_wait_probe(int* status, uint64_t timeout_ns, cudaStream_t s);
+// Dense tensor-pipe rate microbenchmark (see bitlinear_tensor_peak); *units
+// receives the number of ns_out entries written.
+cudaError_t launch_tensor_peak(int kind, int iters, unsigned long long* ns_out, int* status,
+                               uint64_t timeout_ns, int* units, cudaStream_t s);
 
 // Driver entry point for cuTensorMapEncodeTiled, resolved once at run time.
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,

@@ -244,6 +244,23 @@ int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_
                       const int32_t* keep4_pos, int64_t n_keep4, uint16_t* out, int* dev_status,
                       bitlinear_stream_t stream);
 
+/*
+ * Measurement helper (not part of the method): the dense tensor-pipe rate of
+ * this GPU in the MMA shapes the GEMMs issue, for roofline denominators.
+ * Launches one CTA pair per two SMs (kind 0, 1) or one CTA per SM (kind 2);
+ * each issues 4 * iters back-to-back tcgen05 MMAs on operands resident in
+ * shared memory (no unpack, no global reads) and writes the device time of
+ * its stream, in ns, to ns_out[unit].
+ *   kind 0: kind::i8, CTA pair, M = 256, N = 256, K = 32 (2 M N K ops each)
+ *   kind 1: kind::mxf4, CTA pair, M = 256, N = 256, K = 64, unit scales
+ *   kind 2: kind::i8, one CTA, M = 128, N = 256, K = 32
+ *   ns_out     device uint64 [SM count] (the first *units_out entries written)
+ *   units_out  host int: CTA pairs (kind 0, 1) or CTAs (kind 2) launched
+ * Rate = units * 4 * iters * 2 M N K / max(ns_out).
+ */
+int bitlinear_tensor_peak(int kind, int iters, uint64_t* ns_out, int* units_out, int* dev_status,
+                          bitlinear_stream_t stream);
+
 /* Synchronise the stream and read *dev_status: BITLINEAR_OK, or
  * BITLINEAR_ERR_TIMEOUT if a kernel gave up a bounded wait. */
 int bitlinear_check_status(const int* dev_status, bitlinear_stream_t stream);

@@ -20,7 +20,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(_lib._SIGS)
-    assert B.version() == 104
+    assert B.version() == 105
 
 
 @pytest.mark.parametrize("K,N,groups,seed", [

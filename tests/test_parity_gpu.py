@@ -349,7 +349,7 @@ def test_gemm_fp4_max_k_extreme_accumulators():
     assert np.array_equal(host(acc).astype(np.float64), want)
 
 
-@pytest.mark.parametrize("M", [1, 64])
+@pytest.mark.parametrize("M", [1, 8, 64])
 def test_gemv_max_k_extreme_codes(M):
     """The decode paths at K = 32768 (CUDA-core for one token, tensor-core for
     64) with codes of -128 against all-+1 / all--1 rows."""
@@ -647,3 +647,14 @@ def test_kv_attention_full_size_planted_edges():
     q = W.normal_bf16(np.random.default_rng(10), (3, 32, 128))
     out = B.kv_attention_3bit(dev_bf16(q), kst, vst, keep)
     _check_attention(q, tuple(host(t) for t in kst), tuple(host(t) for t in vst), (0,), out=out)
+
+
+def test_tensor_peak_measures_the_pipe():
+    """The measurement helper runs every kind without a timeout and reports
+    rates in the range a B200's tensor pipe can give (dense int8 near
+    4.5 POPS nominal, block-scaled FP4 near 9)."""
+    r = {k: B.tensor_peak(k, 512) for k in (0, 1, 2)}
+    B.check_status()
+    assert r[0]["units"] * 2 == r[2]["units"] // 2 * 2 and r[0]["units"] >= 1
+    assert 1000 < r[0]["tops"] < 6000 and 1000 < r[2]["tops"] < 6000
+    assert 2000 < r[1]["tops"] < 12000
