@@ -1,4 +1,4 @@
-// Decode-time BitLinear for 1..8 tokens on the warp-level tensor-core path
+// Decode-time BitLinear for 2..8 tokens on the warp-level tensor-core path
 // (mma.sync m16n8k32, unsigned 8-bit weight codes x signed 8-bit activations,
 // int32 accumulate).
 //
@@ -32,23 +32,25 @@
 // Inside one MMA the k order is free as long as A and B agree: for lane
 // (g = lane / 4, c = lane % 4) the fragment registers a0 / a2 (rows g) and
 // b0 / b1 (token g) hold the same four physical elements each: elements
-// {0,2,4,6} and {8,10,12,14} (or {1,3,5,7} and {9,11,13,15}) of the lane's
-// word. Lane c of a warp takes words 2c and 2c+1 of a 128-deep k span.
+// {0,2,4,6} and {8,10,12,14} (or {1,3,5,7} and {9,11,13,15}) of one word.
+// In a 256-deep k chunk (64 bytes of a row) lane c takes the four words
+// 4c .. 4c+3 (one 16-byte load per row), and two MMAs per word cover it.
 //
 // Data flow. Each CTA owns a contiguous range of R output rows (a multiple of
 // 8, equal up to 8 rows over the grid, so the weight bytes per SM are
-// balanced), processed in blocks of 16 rows. A block arrives as one bulk
-// copy per row (the row's K/4 contiguous bytes, every lane of a warp issuing
-// one), into a shared-memory slot with a row pitch of K/4 + 16 bytes: the
-// padding spreads the rows of an MMA fragment over all 32 banks. The slots
-// form a ring; the first ones are requested before the kernel waits for the
-// previous one in the stream (the weights do not depend on it), and the CTA
-// needs under half an SM, so the next kernel's CTAs sit beside it and stream
-// their weights while this one computes. The activation rows are staged the
-// same way after the wait. All eight consumer warps work on every block,
-// each on its own 128-deep spans of K (four independent accumulators per
-// span keep the MMAs overlapped), and add their partial sums into a small
-// shared-memory array with atomics; the epilogue reads it once.
+// balanced), processed in blocks of 16 rows. A block is 16 consecutive rows
+// of the packed weights, one contiguous range, so it arrives by a single
+// bulk copy into a shared-memory slot (the copy engine's cost is per request,
+// and a request per row would throttle it). The slots form a ring; the first
+// ones are requested before the kernel waits for the previous one in the
+// stream (the weights do not depend on it), and the CTA needs under half an
+// SM, so the next kernel's CTAs sit beside it and stream their weights while
+// this one computes. The activation rows are staged after the wait and, when
+// every warp's share of K is at most two chunks, regrouped once into
+// registers for all blocks. All eight consumer warps work on every block,
+// each on its own chunks of K (four independent accumulators), and add their
+// partial sums into a small shared-memory array with atomics; the epilogue
+// reads it once.
 //   warps 0-7  consumers (masks, MMAs)
 //   warp  8    copies: activation rows, row and group scales, ring refills
 // Rows of a 16-row block past R are never copied; their results are
@@ -66,15 +68,15 @@ constexpr int WARPS = 8;                   // consumer warps
 constexpr int THREADS = (WARPS + 1) * 32;  // + the copy warp
 constexpr int SMEM_CTA = 110 * 1024;       // two CTAs fit on one SM
 constexpr int MAX_ROWS = 160;              // rows per CTA (10 blocks)
+constexpr int XREG_CHUNKS = 2;             // chunks per warp whose activations stay in registers
 
 struct Params {
   int M, N, K;
-  int nspan;       // 128-deep spans of K
+  int nchunk;      // 256-deep chunks of K (the last may be 128 deep)
   int NB;          // 16-row blocks of the largest CTA
   int S;           // ring slots (blocks)
   int n8;          // N / 8
-  int pitch;       // weight row pitch in shared memory: K / 4 + 16
-  int x_pitch;     // activation row pitch: K + 16
+  int x_pitch;     // activation row pitch in shared memory: K + 16
   int x_off;       // offsets of the shared-memory regions
   int part_off;
   int bar_off;
@@ -93,8 +95,7 @@ struct Params {
 // D (16 x 8, s32) += A (16 x 32, u8) * B (32 x 8, s8)
 __device__ __forceinline__ void mma_u8s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
                                          uint32_t a3, uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+  asm("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
       "{%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -123,15 +124,23 @@ __device__ __forceinline__ int byte_sum(uint4 v) {
   return __dp4a(static_cast<int>(v.w), 0x01010101, s);
 }
 
-// MMA row g of a 16-row block <-> block row sigma(g) (and 8 + sigma(g)): a
-// 16-lane phase of 8-byte shared loads then touches rows {0,2,4,6} (or
-// {1,3,5,7}), which the padded pitch places on disjoint banks.
-__device__ __forceinline__ int sigma(int g) { return ((g & 3) << 1) | (g >> 2); }
+// The two MMAs of one packed word per row: scale-1 and scale-16 fields of
+// word wa (MMA row g) and wb (row g + 8) against the regrouped activations.
+__device__ __forceinline__ void word_mma(int (&acc1)[4], int (&acc16)[4], uint32_t wa, uint32_t wb,
+                                         const uint4& x) {
+  const uint32_t ta = wa >> 2, tb = wb >> 2;
+  mma_u8s8(acc1, wa & 0x03030303u, wb & 0x03030303u, ta & 0x03030303u, tb & 0x03030303u, x.x, x.y);
+  mma_u8s8(acc16, wa & 0x30303030u, wb & 0x30303030u, ta & 0x30303030u, tb & 0x30303030u, x.z, x.w);
+}
 
+// XREG: every warp has at most XREG_CHUNKS chunks, whose regrouped
+// activations are loaded once and kept in registers for all blocks.
+template <bool XREG>
 __global__ void __launch_bounds__(THREADS, 2) bitlinear_gemv_mma_kernel(const Params p) {
   extern __shared__ __align__(16) uint8_t smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int SLOT = 16 * p.pitch;
+  const int row_bytes = p.K >> 2;
+  const int SLOT = 16 * row_bytes;
   uint8_t* xsm = smem + p.x_off;                                    // [M][x_pitch] activation codes
   int32_t* part = reinterpret_cast<int32_t*>(smem + p.part_off);    // [NB][16][8] sums over warps
   float* xs_s = reinterpret_cast<float*>(part + p.NB * 128);        // [8] row scales
@@ -146,7 +155,6 @@ __global__ void __launch_bounds__(THREADS, 2) bitlinear_gemv_mma_kernel(const Pa
   const int r0 = 8 * oct_lo;
   const int R = 8 * (oct_hi - oct_lo);
   const int nblocks = (R + 15) >> 4;
-  const uint32_t row_bytes = static_cast<uint32_t>(p.K >> 2);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < p.S; ++i) {
@@ -165,20 +173,18 @@ __global__ void __launch_bounds__(THREADS, 2) bitlinear_gemv_mma_kernel(const Pa
     *s_abort = 1;
     report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
   };
-  // block b into slot b % S: lane i < rows of the block copies row i (the
-  // whole warp calls this; lane 0 announces the bytes first)
+  // block b (rows r0 + 16 b .. , one contiguous range) into slot b % S
   auto issue_block = [&](int b) {
-    const int rows = min(16, R - 16 * b);
+    const uint32_t bytes = static_cast<uint32_t>(min(16, R - 16 * b) * row_bytes);
     uint64_t* bar = &full[b % p.S];
-    if (lane == 0) mbar_arrive_expect_tx(bar, static_cast<uint32_t>(rows) * row_bytes);
-    __syncwarp();
-    if (lane < rows)
-      bulk_load_1d(smem_u32(smem + (b % p.S) * SLOT + lane * p.pitch),
-                   p.Wp + static_cast<int64_t>(r0 + 16 * b + lane) * row_bytes, row_bytes, bar);
+    mbar_arrive_expect_tx(bar, bytes);
+    bulk_load_1d(smem_u32(smem + (b % p.S) * SLOT), p.Wp + static_cast<int64_t>(r0 + 16 * b) * row_bytes,
+                 bytes, bar);
   };
 
   // the first blocks of the ring, one warp each, before the dependency wait
-  for (int b = warp; b < nblocks && b < p.S; b += WARPS + 1) issue_block(b);
+  if (lane == 0)
+    for (int b = warp; b < nblocks && b < p.S; b += WARPS + 1) issue_block(b);
 
   if (warp == WARPS) {
     // ------------------------------------------------------------ copies
@@ -191,18 +197,17 @@ __global__ void __launch_bounds__(THREADS, 2) bitlinear_gemv_mma_kernel(const Pa
       xs_s[lane] = __ldg(p.xs + lane);
     }
     if (lane < p.G) gam_s[lane] = __ldg(p.gamma + lane);
-    int b = p.S;
-    for (; b < nblocks; ++b) {
-      // the slot's previous block has been consumed by all eight warps
-      const bool got = mbar_wait(&empty[b % p.S], ((b / p.S) - 1) & 1, tmo, s_abort);
-      if (!__all_sync(0xFFFFFFFFu, got)) {
-        if (lane == 0) fail();
-        break;
-      }
-      issue_block(b);
-    }
-    // do not leave while copies into this CTA's shared memory are in flight
     if (lane == 0) {
+      int b = p.S;
+      for (; b < nblocks; ++b) {
+        // the slot's previous block has been consumed by all eight warps
+        if (!mbar_wait(&empty[b % p.S], ((b / p.S) - 1) & 1, tmo, s_abort)) {
+          fail();
+          break;
+        }
+        issue_block(b);
+      }
+      // do not leave while copies into this CTA's shared memory are in flight
       for (int d = 0, j = min(b, nblocks) - 1; d < p.S && j >= 0; ++d, --j)
         mbar_wait(&full[j % p.S], (j / p.S) & 1, tmo, nullptr);
       mbar_wait(xbar, 0, tmo, nullptr);
@@ -210,54 +215,87 @@ __global__ void __launch_bounds__(THREADS, 2) bitlinear_gemv_mma_kernel(const Pa
   } else {
     // ---------------------------------------------------------- consumers
     const int g = lane >> 2, c = lane & 3;
-    const int ra = sigma(g), rb = ra + 8;  // block rows of MMA rows g, g + 8
-    const bool tok = g < p.M;
-    const uint32_t xrow = smem_u32(xsm) + g * p.x_pitch + 32 * c;    // + 128 sp: token g's span bytes
-    const int qa = ra * p.pitch + 8 * c, qb = rb * p.pitch + 8 * c;  // + 32 sp: the lane's words
+    const int rows_a = (((g & 3) << 1) | (g >> 2));  // block row of MMA row g (rows {0,2,4,6} share a
+    const int rows_b = rows_a + 8;                    // half-warp phase of the 16-byte loads)
+    const int gx = g < p.M ? g : 0;                   // lanes of absent tokens read row 0 and zero it
+    const uint8_t* xrow = xsm + gx * p.x_pitch + 64 * c;  // + 256 chunk: this lane's 64 bytes
     bool ok = mbar_wait(xbar, 0, tmo, s_abort);
     if (!ok) fail();
-    int xsum = 0;  // sum of token g's codes over this warp's spans
+    // this warp's chunks: warp, warp + 8, ...; a chunk's activations as four
+    // regrouped 16-byte groups (token g, k = 256 chunk + 64 c .. + 63)
+    auto load_x = [&](int ch, uint4 (&xv)[4], int& xsum) {
+      const int kbytes = min(256, p.K - 256 * ch);  // 256, or 128 for a short last chunk
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (64 * c + 16 * i < kbytes) v = *reinterpret_cast<const uint4*>(xrow + 256 * ch + 16 * i);
+        if (g >= p.M) v = make_uint4(0u, 0u, 0u, 0u);
+        xsum += byte_sum(v);
+        xv[i] = regroup16(v);
+      }
+    };
+    uint4 xr[XREG ? XREG_CHUNKS : 1][4];
+    int xsum = 0;
+    if constexpr (XREG) {
+#pragma unroll
+      for (int j = 0; j < XREG_CHUNKS; ++j) {
+        const int ch = warp + WARPS * j;
+        if (ch < p.nchunk) load_x(ch, xr[j], xsum);
+        else {
+#pragma unroll
+          for (int i = 0; i < 4; ++i) xr[j][i] = make_uint4(0u, 0u, 0u, 0u);
+        }
+      }
+    }
     for (int b = 0; ok && b < nblocks; ++b) {
       const int slot = b % p.S;
       if (!mbar_wait(&full[slot], (b / p.S) & 1, tmo, s_abort)) {
         fail();
         break;
       }
-      const uint32_t tile = smem_u32(smem + slot * SLOT);
-      int a1[4] = {0, 0, 0, 0}, a16[4] = {0, 0, 0, 0}, b1[4] = {0, 0, 0, 0}, b16[4] = {0, 0, 0, 0};
-#pragma unroll 2
-      for (int sp = warp; sp < p.nspan; sp += WARPS) {
-        uint4 xv0 = make_uint4(0u, 0u, 0u, 0u), xv1 = xv0;
-        if (tok) {
-          xv0 = ld_shared_v4(xrow + 128 * sp);
-          xv1 = ld_shared_v4(xrow + 128 * sp + 16);
+      const uint8_t* tile = smem + slot * SLOT;
+      const uint8_t* pa = tile + rows_a * row_bytes + 16 * c;
+      const uint8_t* pb = tile + rows_b * row_bytes + 16 * c;
+      int e1[4] = {0, 0, 0, 0}, e16[4] = {0, 0, 0, 0}, o1[4] = {0, 0, 0, 0}, o16[4] = {0, 0, 0, 0};
+      auto chunk = [&](int ch, const uint4 (&xv)[4]) {
+        // words 4c .. 4c+3 of the chunk's 64 bytes of rows a and b (zero past K)
+        uint4 wa = make_uint4(0u, 0u, 0u, 0u), wb = wa;
+        if (256 * ch + 64 * c < p.K) {
+          wa = *reinterpret_cast<const uint4*>(pa + 64 * ch);
+          wb = *reinterpret_cast<const uint4*>(pb + 64 * ch);
         }
-        if (b == 0) xsum += byte_sum(xv0) + byte_sum(xv1);
-        const uint4 x0 = regroup16(xv0), x1 = regroup16(xv1);
-        const uint2 wa = ld_shared_v2(tile + qa + 32 * sp);
-        const uint2 wb = ld_shared_v2(tile + qb + 32 * sp);
-        const uint32_t ta0 = wa.x >> 2, tb0 = wb.x >> 2, ta1 = wa.y >> 2, tb1 = wb.y >> 2;
-        // word 2c of the span (wa.x / wb.x) and word 2c + 1, scales 1 and 16
-        mma_u8s8(a1, wa.x & 0x03030303u, wb.x & 0x03030303u, ta0 & 0x03030303u, tb0 & 0x03030303u, x0.x, x0.y);
-        mma_u8s8(a16, wa.x & 0x30303030u, wb.x & 0x30303030u, ta0 & 0x30303030u, tb0 & 0x30303030u, x0.z, x0.w);
-        mma_u8s8(b1, wa.y & 0x03030303u, wb.y & 0x03030303u, ta1 & 0x03030303u, tb1 & 0x03030303u, x1.x, x1.y);
-        mma_u8s8(b16, wa.y & 0x30303030u, wb.y & 0x30303030u, ta1 & 0x30303030u, tb1 & 0x30303030u, x1.z, x1.w);
+        word_mma(e1, e16, wa.x, wb.x, xv[0]);
+        word_mma(o1, o16, wa.y, wb.y, xv[1]);
+        word_mma(e1, e16, wa.z, wb.z, xv[2]);
+        word_mma(o1, o16, wa.w, wb.w, xv[3]);
+      };
+      if constexpr (XREG) {
+#pragma unroll
+        for (int j = 0; j < XREG_CHUNKS; ++j)
+          if (warp + WARPS * j < p.nchunk) chunk(warp + WARPS * j, xr[j]);
+      } else {
+        for (int ch = warp; ch < p.nchunk; ch += WARPS) {
+          uint4 xv[4];
+          int xs_unused = 0;
+          load_x(ch, xv, b == 0 ? xsum : xs_unused);
+          chunk(ch, xv);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[slot]);  // this warp is done with the slot
       if (b == 0) {
-        // token sums over this warp's spans: lanes of group g hold token g's
+        // token sums over this warp's chunks: lanes of group g hold token g's
         xsum += __shfl_xor_sync(0xFFFFFFFFu, xsum, 1);
         xsum += __shfl_xor_sync(0xFFFFFFFFu, xsum, 2);
       }
       // D columns 2c, 2c + 1 are tokens 2c, 2c + 1: their sums sit in lanes 8c and 8c + 4
       const int s0 = __shfl_sync(0xFFFFFFFFu, xsum, 8 * c);
       const int s1 = __shfl_sync(0xFFFFFFFFu, xsum, 8 * c + 4);
-      int32_t* pb = part + b * 128;
-      atomicAdd(&pb[ra * 8 + 2 * c], a1[0] + b1[0] + ((a16[0] + b16[0]) >> 4) - s0);
-      atomicAdd(&pb[ra * 8 + 2 * c + 1], a1[1] + b1[1] + ((a16[1] + b16[1]) >> 4) - s1);
-      atomicAdd(&pb[rb * 8 + 2 * c], a1[2] + b1[2] + ((a16[2] + b16[2]) >> 4) - s0);
-      atomicAdd(&pb[rb * 8 + 2 * c + 1], a1[3] + b1[3] + ((a16[3] + b16[3]) >> 4) - s1);
+      int32_t* pp = part + b * 128;
+      atomicAdd(&pp[rows_a * 8 + 2 * c], e1[0] + o1[0] + ((e16[0] + o16[0]) >> 4) - s0);
+      atomicAdd(&pp[rows_a * 8 + 2 * c + 1], e1[1] + o1[1] + ((e16[1] + o16[1]) >> 4) - s1);
+      atomicAdd(&pp[rows_b * 8 + 2 * c], e1[2] + o1[2] + ((e16[2] + o16[2]) >> 4) - s0);
+      atomicAdd(&pp[rows_b * 8 + 2 * c + 1], e1[3] + o1[3] + ((e16[3] + o16[3]) >> 4) - s1);
     }
   }
   pdl_wait();       // the previous kernel may still read y
@@ -287,8 +325,7 @@ struct GemvMmaLayout {
 };
 static GemvMmaLayout gemv_mma_layout(int S, int NB, int M, int K) {
   GemvMmaLayout L;
-  const int pitch = K / 4 + 16;
-  L.x_off = S * 16 * pitch;
+  L.x_off = S * 16 * (K / 4);
   L.part_off = L.x_off + M * (K + 16);
   L.bar_off = L.part_off + NB * 128 * 4 + 16 * 4;
   L.total = L.bar_off + 8 * (2 * S + 1) + 16;
@@ -308,14 +345,13 @@ cudaError_t launch_gemv_mma(const GemmArgs& a, cudaStream_t s, const char** why)
   p.M = static_cast<int>(a.M);
   p.N = static_cast<int>(a.N);
   p.K = static_cast<int>(a.K);
-  p.nspan = p.K / 128;
+  p.nchunk = (p.K + 255) / 256;
   p.n8 = p.N / 8;
   // one CTA per SM (two fit on one), at most MAX_ROWS rows each
   int grid = std::min(num_sms(), p.n8);
   grid = std::max(grid, (p.n8 + MAX_ROWS / 8 - 1) / (MAX_ROWS / 8));
   const int r_hi = 8 * ((p.n8 + grid - 1) / grid);
   p.NB = (r_hi + 15) / 16;
-  p.pitch = p.K / 4 + 16;
   p.x_pitch = p.K + 16;
   // as many slots as leave room for a second CTA on the SM (the next
   // kernel's), at least two
@@ -339,10 +375,12 @@ cudaError_t launch_gemv_mma(const GemmArgs& a, cudaStream_t s, const char** why)
   p.ldy = a.ldo;
   p.status = a.status;
   p.timeout_ns = a.timeout_ns;
-  cudaError_t e = set_smem_limit(bitlinear_gemv_mma_kernel, L.total, true);
+  const bool xreg = p.nchunk <= WARPS * XREG_CHUNKS;
+  void (*kern)(Params) = xreg ? bitlinear_gemv_mma_kernel<true> : bitlinear_gemv_mma_kernel<false>;
+  cudaError_t e = set_smem_limit(kern, L.total, true);
   if (e != cudaSuccess) return e;
-  return launch_kernel(bitlinear_gemv_mma_kernel, dim3(static_cast<unsigned>(grid)), dim3(THREADS),
-                       static_cast<size_t>(L.total), s, 0u, p);
+  return launch_kernel(kern, dim3(static_cast<unsigned>(grid)), dim3(THREADS), static_cast<size_t>(L.total), s,
+                       0u, p);
 }
 
 }  // namespace blt
