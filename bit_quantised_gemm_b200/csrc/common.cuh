@@ -33,6 +33,18 @@ __device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi
   return min(max(c, static_cast<int>(lo)), static_cast<int>(hi));
 }
 
+// v <- fl(fl(v * s) + bias) for both values: two IEEE roundings each. The
+// products come from one paired fp32 multiply; the adds stay scalar IEEE adds,
+// which are never contracted with it into a fused multiply-add (a fused
+// x * s + bias rounds once and can land on the other integer at a .5 tie).
+__device__ __forceinline__ void mul_then_add_rn(float& lo, float& hi, float s, float bias) {
+  asm("{\n\t.reg .b64 x, m;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 m, {%2, %2};\n\t"
+      "mul.rn.f32x2 x, x, m;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(lo), "+f"(hi) : "f"(s));
+  lo = __fadd_rn(lo, bias);
+  hi = __fadd_rn(hi, bias);
+}
+
 __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {
   return (static_cast<uint32_t>(a) & 0xFFu) | ((static_cast<uint32_t>(b) & 0xFFu) << 8) |
          ((static_cast<uint32_t>(c) & 0xFFu) << 16) | ((static_cast<uint32_t>(d) & 0xFFu) << 24);

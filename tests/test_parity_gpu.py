@@ -104,6 +104,30 @@ def test_topk_parity(K, k):
     assert np.array_equal(host(xs), xs_o)
 
 
+@pytest.mark.parametrize("K", [16, 272, 528, 1040, 2064, 4096])
+def test_topk_extreme_rows(K):
+    """Rows whose selection takes the rarer routes: a threshold far below the
+    row maximum (wide dynamic range, a lone outlier, mostly zeros), every
+    finite bf16 bit pattern, subnormal-only rows, k = 1 and k = K; one
+    column count per lane width, M not a multiple of the rows per block."""
+    rng = np.random.default_rng(K)
+    M = 7
+    xf = rng.standard_normal((M, K)).astype(np.float32)
+    xf[0] = np.exp(rng.uniform(-80, 80, K)) * np.sign(rng.standard_normal(K))
+    xf[1] *= 1e-3
+    xf[1, K // 3] = 1e30
+    xf[2, : K - K // 8] = 0.0
+    x = O.f32_to_bf16(xf)
+    x[3] = rng.integers(0, 0x7F80, K).astype(np.uint16) | (rng.integers(0, 2, K).astype(np.uint16) << 15)
+    x[4] = rng.integers(0, 0x80, K).astype(np.uint16) | (rng.integers(0, 2, K).astype(np.uint16) << 15)
+    for kk in (1, K // 2, K - 1, K):
+        q, xs, mask = B.topk_sparsify_i8(dev_bf16(x), k=kk, mask=True)
+        q_o, xs_o, m_o = O.topk_sparsify_i8(x, kk)
+        assert np.array_equal(host(mask), O.pack_mask_bits(m_o)), kk
+        assert np.array_equal(host(q), q_o), kk
+        assert np.array_equal(host(xs), xs_o), kk
+
+
 def test_topk_full_size_o_proj():
     d = W.o_proj_sparse(make_weights=False, M=1024)  # the o_proj input recipe, 1024 rows
     q, xs, mask = B.topk_sparsify_i8(dev_bf16(d["x"]), mask=True)
