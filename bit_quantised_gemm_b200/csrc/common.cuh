@@ -38,11 +38,9 @@ __device__ __forceinline__ int quant_code(float h, float inv, float lo, float hi
 // which are never contracted with it into a fused multiply-add (a fused
 // x * s + bias rounds once and can land on the other integer at a .5 tie).
 __device__ __forceinline__ void mul_then_add_rn(float& lo, float& hi, float s, float bias) {
-  asm("{\n\t.reg .b64 x, m;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 m, {%2, %2};\n\t"
-      "mul.rn.f32x2 x, x, m;\n\tmov.b64 {%0, %1}, x;\n\t}"
-      : "+f"(lo), "+f"(hi) : "f"(s));
-  lo = __fadd_rn(lo, bias);
-  hi = __fadd_rn(hi, bias);
+  const float2 p = __fmul2_rn(make_float2(lo, hi), make_float2(s, s));
+  lo = __fadd_rn(p.x, bias);
+  hi = __fadd_rn(p.y, bias);
 }
 
 __device__ __forceinline__ uint32_t pack_s8x4(int a, int b, int c, int d) {

@@ -635,7 +635,11 @@ def _check_attention(q, ks, vs, keep, out=None):
 @pytest.mark.parametrize("Bq,H,D,T,keep", [
     (1, 4, 128, 1, (0,)), (1, 4, 128, 37, ()), (3, 4, 128, 300, (0, 5, 130)), (8, 4, 256, 513, (0,)),
     (11, 8, 128, 1000, (0, 999)), (1, 4, 128, 4096, (0,)), (2, 4, 128, 129, tuple(range(0, 129, 3))),
-    (1, 4, 256, 2000, ())])
+    (1, 4, 256, 2000, ()),
+    # one query per head at D = 128 (the warp-per-32-tokens kernel): 4-bit tokens on warp and tile
+    # edges, many 4-bit tokens, token counts that split unevenly over the cluster
+    (1, 8, 128, 1000, (0, 31, 32, 255, 256, 511, 999)), (1, 4, 128, 2049, tuple(range(0, 2049, 7))),
+    (1, 4, 128, 8191, (0, 4095, 8190))])
 def test_kv_attention_parity(Bq, H, D, T, keep):
     q, ks, vs = _attn_case(np.random.default_rng(Bq * 100 + T), Bq, H, D, T, keep)
     _check_attention(q, ks, vs, keep)
@@ -654,7 +658,8 @@ def test_kv_attention_full_size(Bq):
     _check_attention(q, tuple(host(t) for t in kst), tuple(host(t) for t in vst), (0,), out=out)
 
 
-def test_kv_attention_full_size_planted_edges():
+@pytest.mark.parametrize("Bq", [1, 3])
+def test_kv_attention_full_size_planted_edges(Bq):
     """Every token at a 32-token boundary (t % 32 in {0, 31}, which includes
     each 256-token tile edge and each split of the tokens over a cluster)
     carries value rows 16x larger, so a boundary token lost or counted twice
@@ -668,7 +673,7 @@ def test_kv_attention_full_size_planted_edges():
     keep = torch.tensor([0], dtype=torch.int32, device=DEV)
     kst = B.kv_quant_3bit(dev_bf16(d["k_cache"]), keep)
     vst = B.kv_quant_3bit(dev_bf16(v_bits), keep)
-    q = W.normal_bf16(np.random.default_rng(10), (3, 32, 128))
+    q = W.normal_bf16(np.random.default_rng(10), (Bq, 32, 128))
     out = B.kv_attention_3bit(dev_bf16(q), kst, vst, keep)
     _check_attention(q, tuple(host(t) for t in kst), tuple(host(t) for t in vst), (0,), out=out)
 
