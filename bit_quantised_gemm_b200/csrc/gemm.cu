@@ -99,6 +99,18 @@ struct Params {
   uint64_t timeout_ns;
 };
 
+// The k-block a tile handles at step kb. With long K (16 k-blocks or more)
+// tile t starts at k-block t mod num_kb, so the CTAs working on different
+// tiles at the same moment read different activation and weight columns:
+// down_proj (K = 11008, 43 k-blocks) 131 -> 121 us; at K = 2048 the order
+// made no difference. The sums are exact in any order (int32, or fp32 sums
+// of multiples of 0.5 below 2^24).
+__device__ __forceinline__ int kb_rotation(int tile, int num_kb) { return num_kb >= 16 ? tile % num_kb : 0; }
+__device__ __forceinline__ int kb_at(int kb, int rot, int num_kb) {
+  const int k = kb + rot;
+  return k >= num_kb ? k - num_kb : k;
+}
+
 template <bool FP4, bool PAIR, bool MX>
 __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -205,7 +217,9 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int tile = cta_slot; ok && tile < p.num_tiles; tile += cta_stride) {
         const int m0 = (tile % p.tiles_m) * TILE_M + static_cast<int>(rank) * BM;
         const int n0 = (tile / p.tiles_m) * BN + static_cast<int>(rank) * L::BROWS;
+        const int rot = kb_rotation(tile, p.num_kb);
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int kg = kb_at(kb, rot, p.num_kb);
           const int S = act ? S_TMA : S_W;
           const uint32_t s = it % S, ph = (it / S) & 1;
           if (!mbar_wait(act ? &empty[s] : &wempty[s], ph ^ 1, tmo, s_abort)) { fail(); ok = false; break; }
@@ -213,14 +227,14 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             uint8_t* dst = smem + L::OFF_A + s * A_BYTES;
             if (PAIR) {  // two 128-byte swizzled chunks (int8: 128 k each, e2m1: 256 k)
               if (leader) mbar_arrive_expect_tx(&afull[s], 2 * A_TX);
-              tma_load_3d_pair(dst, &tmA, lead(&afull[s]), 0, m0, kb * L::KSUB);
+              tma_load_3d_pair(dst, &tmA, lead(&afull[s]), 0, m0, kg * L::KSUB);
             } else {
               mbar_arrive_expect_tx(&afull[s], A_TX);
-              tma_load_2d(dst, &tmA, &afull[s], kb * BK, m0);
+              tma_load_2d(dst, &tmA, &afull[s], kg * BK, m0);
             }
           } else {
             mbar_arrive_expect_tx(&wfull[s], L::WP_BYTES);
-            tma_load_2d(smem + L::OFF_WP + s * L::WP_BYTES, &tmW, &wfull[s], kb * (BK / 4), n0);
+            tma_load_2d(smem + L::OFF_WP + s * L::WP_BYTES, &tmW, &wfull[s], kg * (BK / 4), n0);
           }
         }
       }
@@ -251,7 +265,9 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                    : mbar_wait(&tempty[acc], aph ^ 1, tmo, s_abort))) { fail(); break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
+        const int rot = kb_rotation(tile, p.num_kb);
         for (int kb = 0; kb < p.num_kb; ++kb, ++it) {
+          const int kg = kb_at(kb, rot, p.num_kb);
           const uint32_t s = it % S_TMA, ph = (it / S_TMA) & 1;
           const uint32_t b = it % S_B, bph = (it / S_B) & 1;
           const bool got = mbar_wait(&afull[s], ph, tmo, s_abort) &&
@@ -266,7 +282,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
             for (int kk = 0; kk < BK / 64; ++kk) {
               const int sub = kk >> 2, k4 = kk & 3;
-              if (sub > 0 && kb * BK + sub * 256 >= p.K) break;
+              if (sub > 0 && kg * BK + sub * 256 >= p.K) break;
               const uint64_t adesc = smem_desc_sw128(sA + s * A_BYTES + sub * SUB);
               const uint64_t bdesc = smem_desc_sw128(sB + b * L::B_BYTES + sub * L::BROWS * 128);
               mma_mxf4_pair(d_tmem, adesc + 2 * k4, bdesc + 2 * k4, idesc, sfa, sfb, (kb | kk) != 0);
