@@ -6,6 +6,6 @@ from ._lib import (  # noqa: F401
     MODE_FP4, MODE_INT4, MODE_INT8, BitlinearError, check_status, debug_wait_timeout,
     gemm_w2a4, gemm_w2a8, gemm_w2a8_acc, gemm_w2fp4, gemm_w2fp4_acc, gemv_w2, gemv_w2_quant,
     header_functions,
-    kv_attention_3bit, kv_keep4_positions, kv_quant_3bit, lib, quant_act, set_launch_overlap, set_wait_timeout_ns, status_buffer, ternarize_pack,
+    kv_attention_3bit, kv_keep4_positions, kv_quant_3bit, kv_quant_3bit_kv, lib, quant_act, set_launch_overlap, set_wait_timeout_ns, status_buffer, ternarize_pack,
     tensor_peak, topk_sparsify_i8, version,
 )

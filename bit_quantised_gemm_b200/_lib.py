@@ -53,6 +53,7 @@ _SIGS = {
     "bitlinear_gemv_w2_quant": ([_P, _P, _I64, _INT, _P, _P, _P, _INT, _I64, _I64, _I64, _P, _I64, _P, _P],
                                 _INT),
     "kv_quant_3bit": ([_P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P], _INT),
+    "kv_quant_3bit_kv": ([_P, _P, _I64, _I64, _I64, _P, _I64, _P, _P, _P, _P, _P, _P, _P], _INT),
     "kv_keep4_positions": ([_P, _I64, _P, _INT, _P, _P, _P], _INT),
     "bitlinear_check_status": ([_P, _P], _INT),
     "bitlinear_tensor_peak": ([_INT, _INT, _P, _P, _P, _P], _INT),
@@ -382,6 +383,36 @@ def kv_quant_3bit(kv: torch.Tensor, keep4_pos: torch.Tensor | None, codes3=None,
     _check(lib().kv_quant_3bit(_ptr(kv), T, H, D, _ptr(keep4_pos), n4, _ptr(codes3), _ptr(codes4),
                                _ptr(scale), _stream(stream)))
     return codes3, codes4, scale
+
+
+def kv_quant_3bit_kv(k: torch.Tensor, v: torch.Tensor, keep4_pos: torch.Tensor | None, k_store=None,
+                     v_store=None, stream=None):
+    """kv_quant_3bit of a layer's K and V in one launch; returns the two
+    (codes3, codes4, scale) triples."""
+    for name, t in (("k", k), ("v", v)):
+        if t.dim() != 3 or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous [T x H x D] tensor")
+        _need(t, name, _BF16_LIKE)
+    if tuple(k.shape) != tuple(v.shape):
+        raise ValueError(f"k {tuple(k.shape)} and v {tuple(v.shape)} must have one shape")
+    T, H, D = k.shape
+    n4 = 0 if keep4_pos is None else keep4_pos.numel()
+    if keep4_pos is not None:
+        _need(keep4_pos, "keep4_pos", (torch.int32,), 1, contiguous=True)
+
+    def store(given):
+        if given is not None:
+            return given
+        c3 = torch.empty((T, H, 3 * D // 8), dtype=torch.uint8, device=k.device)
+        c4 = torch.empty((n4, H, D // 2), dtype=torch.uint8, device=k.device) if n4 else None
+        return c3, c4, torch.empty((T, H), dtype=torch.float32, device=k.device)
+    ks, vs = store(k_store), store(v_store)
+    _check_kv_store("k ", *ks, T, H, D, n4)
+    _check_kv_store("v ", *vs, T, H, D, n4)
+    _require_cuda(k, v, keep4_pos, *ks, *vs)
+    _check(lib().kv_quant_3bit_kv(_ptr(k), _ptr(v), T, H, D, _ptr(keep4_pos), n4, _ptr(ks[0]), _ptr(ks[1]),
+                                  _ptr(ks[2]), _ptr(vs[0]), _ptr(vs[1]), _ptr(vs[2]), _stream(stream)))
+    return ks, vs
 
 
 def kv_keep4_positions(token_ids: torch.Tensor, special_ids, stream=None) -> torch.Tensor:

@@ -150,7 +150,7 @@ extern "C" {
 
 const char* bitlinear_last_error(void) { return g_err; }
 
-int bitlinear_version(void) { return 105; }
+int bitlinear_version(void) { return 106; }
 
 int bitlinear_set_launch_overlap(int enable) {
   g_overlap.store(enable != 0);
@@ -351,21 +351,44 @@ int bitlinear_gemv_w2_quant(const uint16_t* x, const uint16_t* up, int64_t ldx, 
   return e == cudaSuccess ? ok() : cuda_fail(e, "gemv_w2_quant");
 }
 
+static int kv_quant_check(const char* fn, const uint16_t* kv, int64_t T, int64_t H, int64_t D,
+                          const int32_t* keep4_pos, int64_t n_keep4, const uint8_t* codes3,
+                          const uint8_t* codes4, const float* scale) {
+  if (T < 0 || H <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: bad sizes", fn);
+  if (D != 64 && D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "%s: D must be 64, 128 or 256", fn);
+  if (n_keep4 < 0 || n_keep4 > T || (n_keep4 > 0 && (!keep4_pos || !codes4)))
+    return fail(BITLINEAR_ERR_INVALID_ARG, "%s: bad 4-bit token list", fn);
+  if (T == 0) return BITLINEAR_OK;
+  if (!kv || !codes3 || !scale) return fail(BITLINEAR_ERR_INVALID_ARG, "%s: null pointer", fn);
+  if (!aligned16(kv) || !aligned16(codes3) || (codes4 && !aligned16(codes4)))
+    return fail(BITLINEAR_ERR_ALIGNMENT, "%s: pointers must be 16-byte aligned", fn);
+  if (T * H * (D / 8) >= (1LL << 32) - 256 || n_keep4 > 0x7FFFFFFF)
+    return fail(BITLINEAR_ERR_UNSUPPORTED, "%s: T * H * D / 8 must stay below 2^32", fn);
+  return BITLINEAR_OK;
+}
+
 int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int32_t* keep4_pos,
                   int64_t n_keep4, uint8_t* codes3, uint8_t* codes4, float* scale,
                   bitlinear_stream_t stream) {
-  if (T < 0 || H <= 0) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: bad sizes");
-  if (D != 64 && D != 128 && D != 256) return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: D must be 64, 128 or 256");
-  if (n_keep4 < 0 || n_keep4 > T || (n_keep4 > 0 && (!keep4_pos || !codes4)))
-    return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: bad 4-bit token list");
+  const int rc = kv_quant_check("kv_quant_3bit", kv, T, H, D, keep4_pos, n_keep4, codes3, codes4, scale);
+  if (rc != BITLINEAR_OK) return rc;
   if (T == 0) return ok();
-  if (!kv || !codes3 || !scale) return fail(BITLINEAR_ERR_INVALID_ARG, "kv_quant_3bit: null pointer");
-  if (!aligned16(kv) || !aligned16(codes3) || (codes4 && !aligned16(codes4)))
-    return fail(BITLINEAR_ERR_ALIGNMENT, "kv_quant_3bit: pointers must be 16-byte aligned");
-  if (T * H * (D / 8) >= (1LL << 32) - 256 || n_keep4 > 0x7FFFFFFF)
-    return fail(BITLINEAR_ERR_UNSUPPORTED, "kv_quant_3bit: T * H * D / 8 must stay below 2^32");
   cudaError_t e = blt::launch_kv_quant(kv, T, H, D, keep4_pos, n_keep4, codes3, codes4, scale, stream);
   return e == cudaSuccess ? ok() : cuda_fail(e, "kv_quant_3bit launch");
+}
+
+int kv_quant_3bit_kv(const uint16_t* k, const uint16_t* v, int64_t T, int64_t H, int64_t D,
+                     const int32_t* keep4_pos, int64_t n_keep4, uint8_t* k_codes3, uint8_t* k_codes4,
+                     float* k_scale, uint8_t* v_codes3, uint8_t* v_codes4, float* v_scale,
+                     bitlinear_stream_t stream) {
+  int rc = kv_quant_check("kv_quant_3bit_kv (K)", k, T, H, D, keep4_pos, n_keep4, k_codes3, k_codes4, k_scale);
+  if (rc != BITLINEAR_OK) return rc;
+  rc = kv_quant_check("kv_quant_3bit_kv (V)", v, T, H, D, keep4_pos, n_keep4, v_codes3, v_codes4, v_scale);
+  if (rc != BITLINEAR_OK) return rc;
+  if (T == 0) return ok();
+  cudaError_t e = blt::launch_kv_quant_pair(k, v, T, H, D, keep4_pos, n_keep4, k_codes3, k_codes4, k_scale,
+                                           v_codes3, v_codes4, v_scale, stream);
+  return e == cudaSuccess ? ok() : cuda_fail(e, "kv_quant_3bit_kv launch");
 }
 
 int kv_keep4_positions(const int32_t* token_ids, int64_t T, const int32_t* special_ids,

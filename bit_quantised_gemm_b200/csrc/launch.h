@@ -22,6 +22,9 @@ cudaError_t launch_keep4_positions(const int32_t* ids, int64_t T, const int32_t*
 cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
                             const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
                             float* scale, cudaStream_t s);
+cudaError_t launch_kv_quant_pair(const uint16_t* k, const uint16_t* v, int64_t T, int64_t H, int64_t D,
+                                 const int32_t* keep4, int64_t n4, uint8_t* k3, uint8_t* k4, float* ks,
+                                 uint8_t* v3, uint8_t* v4, float* vs, cudaStream_t s);
 
 // Epilogue of the GEMM kernels.
 enum OutMode : int { kOutBf16 = 0, kOutRaw = 1 };

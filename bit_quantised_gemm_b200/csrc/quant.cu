@@ -756,10 +756,22 @@ constexpr uint32_t kKv3Bias2 = kv3_bias(22, 31, 64);  // fields 22..31
 constexpr int kKeepSmem = 1024;
 constexpr int kKvThreads = 256;
 
+// One launch quantises one or two tensors of the same shape (K and V of a
+// layer): tile t of the 2 ntiles belongs to tensor t / ntiles.
+struct KvSet {
+  const uint16_t* kv;
+  uint8_t* codes3;
+  uint8_t* codes4;
+  float* scale;
+};
+struct KvSets {
+  KvSet s[2];
+  int n;
+};
+
 template <int GP>
 __global__ void __launch_bounds__(kKvThreads, 4) kv_quant_kernel(
-    const uint16_t* __restrict__ kv, uint32_t rows, uint32_t H, const int32_t* __restrict__ keep4,
-    int n4, uint8_t* __restrict__ codes3, uint8_t* __restrict__ codes4, float* __restrict__ scale) {
+    const KvSets sets, uint32_t rows, uint32_t H, const int32_t* __restrict__ keep4, int n4) {
   pdl_wait();  // inputs come from the previous kernel in the stream
   pdl_trigger();
   constexpr int D = 32 * GP;
@@ -770,21 +782,28 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_quant_kernel(
   for (int i = threadIdx.x; i < n4s; i += kKvThreads) s_keep[i] = __ldg(keep4 + i);
   __syncthreads();
   const int g = lane % GP;
-  const uint32_t ntiles = (rows + RPT - 1) / RPT;
+  const uint32_t ntiles = (rows + RPT - 1) / RPT;  // per tensor
+  const uint32_t total = ntiles * static_cast<uint32_t>(sets.n);
   const uint32_t nwarps = gridDim.x * (kKvThreads / 32);
 
-  auto load = [&](uint32_t tile, uint4 (&b)[4]) {
-    const uint32_t row = tile * RPT + lane / GP;
+  auto load = [&](uint32_t gt, uint4 (&b)[4]) {
+    const int set = gt >= ntiles ? 1 : 0;
+    const uint32_t row = (gt - (set ? ntiles : 0u)) * RPT + lane / GP;
 #pragma unroll
     for (int i = 0; i < 4; ++i) b[i] = make_uint4(0u, 0u, 0u, 0u);
     if (row < rows) {
-      const uint4* src = reinterpret_cast<const uint4*>(kv + static_cast<size_t>(row) * D) + 4 * g;
+      const uint16_t* kvp = set ? sets.s[1].kv : sets.s[0].kv;
+      const uint4* src = reinterpret_cast<const uint4*>(kvp + static_cast<size_t>(row) * D) + 4 * g;
 #pragma unroll
       for (int i = 0; i < 4; ++i) b[i] = __ldg(src + i);
     }
   };
-  auto quantise = [&](uint32_t tile, const uint4 (&b)[4]) {
-    const uint32_t row = tile * RPT + lane / GP;
+  auto quantise = [&](uint32_t gt, const uint4 (&b)[4]) {
+    const int set = gt >= ntiles ? 1 : 0;
+    uint8_t* __restrict__ codes3 = set ? sets.s[1].codes3 : sets.s[0].codes3;
+    uint8_t* __restrict__ codes4 = set ? sets.s[1].codes4 : sets.s[0].codes4;
+    float* __restrict__ scale = set ? sets.s[1].scale : sets.s[0].scale;
+    const uint32_t row = (gt - (set ? ntiles : 0u)) * RPT + lane / GP;
     const bool valid = row < rows;
     const uint32_t w[16] = {b[0].x, b[0].y, b[0].z, b[0].w, b[1].x, b[1].y, b[1].z, b[1].w,
                             b[2].x, b[2].y, b[2].z, b[2].w, b[3].x, b[3].y, b[3].z, b[3].w};
@@ -857,26 +876,25 @@ __global__ void __launch_bounds__(kKvThreads, 4) kv_quant_kernel(
 
   uint32_t tile = blockIdx.x * (kKvThreads / 32) + wid;
   uint4 A[4], B[4];
-  if (tile < ntiles) load(tile, A);
-  while (tile < ntiles) {
+  if (tile < total) load(tile, A);
+  while (tile < total) {
     uint32_t nt = tile + nwarps;
-    if (nt < ntiles) load(nt, B);
+    if (nt < total) load(nt, B);
     quantise(tile, A);
     tile = nt;
-    if (tile >= ntiles) break;
+    if (tile >= total) break;
     nt = tile + nwarps;
-    if (nt < ntiles) load(nt, A);
+    if (nt < total) load(nt, A);
     quantise(tile, B);
     tile = nt;
   }
 }
 
-cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
-                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
-                            float* scale, cudaStream_t s) {
+static cudaError_t launch_kv_sets(const KvSets& sets, int64_t T, int64_t H, int64_t D, const int32_t* keep4,
+                                  int64_t n4, cudaStream_t s) {
   const uint32_t rows = static_cast<uint32_t>(T * H);  // the entry point bounds rows * D / 8 < 2^32
   const int GP = static_cast<int>(D / 32);
-  const uint64_t tiles = (static_cast<uint64_t>(rows) * GP + 31) / 32;
+  const uint64_t tiles = static_cast<uint64_t>(sets.n) * ((static_cast<uint64_t>(rows) * GP + 31) / 32);
   const int n = static_cast<int>(n4);
   const uint32_t h = static_cast<uint32_t>(H);
   auto go = [&](auto kern) {
@@ -886,12 +904,31 @@ cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
     const uint64_t want = (tiles + kKvThreads / 32 - 1) / (kKvThreads / 32);
     const uint64_t cap = static_cast<uint64_t>(num_sms()) * static_cast<uint64_t>(per_sm > 0 ? per_sm : 1);
     const unsigned grid = static_cast<unsigned>(want < cap ? want : cap);
-    return launch_kernel(kern, dim3(grid), dim3(kKvThreads), 0, s, 0u, kv, rows, h, keep4, n,
-                         codes3, codes4, scale);
+    return launch_kernel(kern, dim3(grid), dim3(kKvThreads), 0, s, 0u, sets, rows, h, keep4, n);
   };
   if (GP == 2) return go(kv_quant_kernel<2>);
   if (GP == 4) return go(kv_quant_kernel<4>);
   return go(kv_quant_kernel<8>);
+}
+
+cudaError_t launch_kv_quant(const uint16_t* kv, int64_t T, int64_t H, int64_t D,
+                            const int32_t* keep4, int64_t n4, uint8_t* codes3, uint8_t* codes4,
+                            float* scale, cudaStream_t s) {
+  KvSets sets{};
+  sets.s[0] = KvSet{kv, codes3, codes4, scale};
+  sets.s[1] = sets.s[0];
+  sets.n = 1;
+  return launch_kv_sets(sets, T, H, D, keep4, n4, s);
+}
+
+cudaError_t launch_kv_quant_pair(const uint16_t* k, const uint16_t* v, int64_t T, int64_t H, int64_t D,
+                                 const int32_t* keep4, int64_t n4, uint8_t* k3, uint8_t* k4, float* ks,
+                                 uint8_t* v3, uint8_t* v4, float* vs, cudaStream_t s) {
+  KvSets sets{};
+  sets.s[0] = KvSet{k, k3, k4, ks};
+  sets.s[1] = KvSet{v, v3, v4, vs};
+  sets.n = 2;
+  return launch_kv_sets(sets, T, H, D, keep4, n4, s);
 }
 
 // ------------------------------------------------ 4-bit token positions

@@ -203,6 +203,19 @@ int kv_quant_3bit(const uint16_t* kv, int64_t T, int64_t H, int64_t D, const int
                   bitlinear_stream_t stream);
 
 /*
+ * The same quantiser ([R] "Эксперименты") applied to the K and the V cache
+ * of a layer in one launch: k_* are written exactly as kv_quant_3bit(k, ...)
+ * would write them, v_* as kv_quant_3bit(v, ...), with one keep4_pos list
+ * for both. Saves the second launch's ramp when both are quantised
+ * together, as in a decoder layer. Same requirements, per tensor, as
+ * kv_quant_3bit; the two tensors may not overlap their outputs.
+ */
+int kv_quant_3bit_kv(const uint16_t* k, const uint16_t* v, int64_t T, int64_t H, int64_t D,
+                     const int32_t* keep4_pos, int64_t n_keep4, uint8_t* k_codes3, uint8_t* k_codes4,
+                     float* k_scale, uint8_t* v_codes3, uint8_t* v_codes4, float* v_scale,
+                     bitlinear_stream_t stream);
+
+/*
  * The positions kept at 4 bits, from the token ids ([R] "Эксперименты": the
  * <bos> and <eos> tokens stay at 4 bits): every t < T whose token_ids[t]
  * equals one of special_ids, in increasing order; the list kv_quant_3bit and

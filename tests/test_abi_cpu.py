@@ -20,7 +20,7 @@ def test_library_exports_every_declared_function():
     for name in declared:
         assert hasattr(L, name), name
     assert set(declared) == set(_lib._SIGS)
-    assert B.version() == 105
+    assert B.version() == 106
 
 
 @pytest.mark.parametrize("K,N,groups,seed", [
@@ -151,6 +151,17 @@ def test_quantiser_argument_errors():
     assert L.kv_quant_3bit(FAKE, 4, 2, 96, None, 0, FAKE, None, FAKE, None) == _lib.ERR_UNSUPPORTED
     assert L.kv_quant_3bit(FAKE, 4, 2, 128, None, 1, FAKE, FAKE, FAKE, None) == _lib.ERR_INVALID_ARG
     assert L.kv_quant_3bit(FAKE, 0, 2, 128, None, 0, FAKE, None, FAKE, None) == _lib.OK
+    # K and V in one launch: each tensor is checked as kv_quant_3bit checks it
+    assert L.kv_quant_3bit_kv(FAKE, FAKE, 4, 2, 96, None, 0, FAKE, None, FAKE, FAKE, None, FAKE,
+                              None) == _lib.ERR_UNSUPPORTED
+    assert L.kv_quant_3bit_kv(FAKE, FAKE, 4, 2, 128, FAKE, 1, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                              None) == _lib.ERR_INVALID_ARG
+    assert L.kv_quant_3bit_kv(FAKE, None, 4, 2, 128, None, 0, FAKE, None, FAKE, FAKE, None, FAKE,
+                              None) == _lib.ERR_INVALID_ARG
+    assert L.kv_quant_3bit_kv(FAKE, FAKE + 8, 4, 2, 128, None, 0, FAKE, None, FAKE, FAKE, None, FAKE,
+                              None) == _lib.ERR_ALIGNMENT
+    assert L.kv_quant_3bit_kv(FAKE, FAKE, 0, 2, 128, None, 0, FAKE, None, FAKE, FAKE, None, FAKE,
+                              None) == _lib.OK
     assert L.bitlinear_set_wait_timeout_ns(0) == _lib.ERR_INVALID_ARG
     msg = L.bitlinear_last_error().decode()
     assert "timeout" in msg
@@ -245,6 +256,16 @@ def test_binding_rejects_malformed_acc_and_kv_tensors():
         B.kv_quant_3bit(kv, keep.long())
     with pytest.raises(ValueError, match="kv: dtype"):
         B.kv_quant_3bit(kv.float(), keep)
+    with pytest.raises(ValueError, match="CUDA"):
+        B.kv_quant_3bit_kv(kv, kv.clone(), keep)
+    with pytest.raises(ValueError, match="one shape"):
+        B.kv_quant_3bit_kv(kv, kv[:8].contiguous(), keep)
+    with pytest.raises(ValueError, match="v: dtype"):
+        B.kv_quant_3bit_kv(kv, kv.float(), keep)
+    with pytest.raises(ValueError, match="v codes3: shape"):
+        B.kv_quant_3bit_kv(kv, kv, keep, v_store=(torch.empty((T, H, D // 4), dtype=torch.uint8),
+                                                 torch.empty((1, H, D // 2), dtype=torch.uint8),
+                                                 torch.empty((T, H), dtype=torch.float32)))
 
     q = torch.zeros((2, H, D), dtype=torch.bfloat16)
     c3 = torch.zeros((T, H, 3 * D // 8), dtype=torch.uint8)

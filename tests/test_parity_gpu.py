@@ -183,6 +183,29 @@ def test_kv_quant_parity(D, keep):
         assert np.array_equal(host(c4), c4_o)
 
 
+@pytest.mark.parametrize("D,T", [(64, 41), (128, 300), (256, 17)])
+def test_kv_quant_pair_parity(D, T):
+    """K and V in one launch: each cache equals the oracle's for that tensor,
+    with the 4-bit tokens shared and ragged tile counts on both halves."""
+    rng = np.random.default_rng(100 + D)
+    H = 5
+    k, v = W.normal_bf16(rng, (T, H, D)), W.normal_bf16(rng, (T, H, D))
+    k[3, 2] = 0
+    v[T - 1, 0] = 0
+    keep = tuple(sorted({0, 1, T // 2, T - 1}))
+    kp = torch.tensor(keep, dtype=torch.int32, device=DEV)
+    (k3, k4, ks), (v3, v4, vs) = B.kv_quant_3bit_kv(dev_bf16(k), dev_bf16(v), kp)
+    for (c3, c4, s), x in (((k3, k4, ks), k), ((v3, v4, vs), v)):
+        c3_o, c4_o, s_o = O.kv_quant_3bit(x, keep)
+        assert np.array_equal(host(s), s_o)
+        assert np.array_equal(host(c3), c3_o)
+        assert np.array_equal(host(c4), c4_o)
+    (k3n, _, ksn), (v3n, _, vsn) = B.kv_quant_3bit_kv(dev_bf16(k), dev_bf16(v), None)
+    for (c3, s), x in (((k3n, ksn), k), ((v3n, vsn), v)):
+        c3_o, _, s_o = O.kv_quant_3bit(x, ())
+        assert np.array_equal(host(s), s_o) and np.array_equal(host(c3), c3_o)
+
+
 # ------------------------------------------------------------------ GEMMs
 def prep_weights(K, N, groups, seed):
     Wm = W.weights(np.random.default_rng(seed), K, N)
