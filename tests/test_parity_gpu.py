@@ -659,10 +659,12 @@ def _check_attention(q, ks, vs, keep, out=None):
     (1, 4, 128, 1, (0,)), (1, 4, 128, 37, ()), (3, 4, 128, 300, (0, 5, 130)), (8, 4, 256, 513, (0,)),
     (11, 8, 128, 1000, (0, 999)), (1, 4, 128, 4096, (0,)), (2, 4, 128, 129, tuple(range(0, 129, 3))),
     (1, 4, 256, 2000, ()),
-    # one query per head at D = 128 (the warp-per-32-tokens kernel): 4-bit tokens on warp and tile
-    # edges, many 4-bit tokens, token counts that split unevenly over the cluster
+    # D = 128 (the tensor-core kernel): 4-bit tokens on warp and tile edges, many 4-bit tokens (up
+    # to the 1024 the entry point takes, several in every warp), token counts that split unevenly
+    # over the cluster, 5 queries (8-query groups with 3 empty) and 12 (a group of 8 and one of 4)
     (1, 8, 128, 1000, (0, 31, 32, 255, 256, 511, 999)), (1, 4, 128, 2049, tuple(range(0, 2049, 7))),
-    (1, 4, 128, 8191, (0, 4095, 8190))])
+    (1, 4, 128, 8191, (0, 4095, 8190)), (2, 4, 128, 4096, tuple(range(0, 4096, 4))),
+    (5, 4, 128, 777, (0, 1, 2, 3, 776)), (12, 4, 128, 300, (0, 150))])
 def test_kv_attention_parity(Bq, H, D, T, keep):
     q, ks, vs = _attn_case(np.random.default_rng(Bq * 100 + T), Bq, H, D, T, keep)
     _check_attention(q, ks, vs, keep)
