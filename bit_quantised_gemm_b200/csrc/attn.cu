@@ -79,6 +79,15 @@ struct Smem {
   int k4_n;
 };
 
+__device__ __forceinline__ void st_dsmem_f32(uint32_t addr, float v) {
+  asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_dsmem_v4f32(uint32_t addr, float4 v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
@@ -454,8 +463,10 @@ struct SmemMQ {
   float wm[MQ_WARPS][QG], wl[MQ_WARPS][QG];
   float wf[MQ_WARPS][QG];             // the warps' merge factors
   float rf[QG][16];                   // the cluster's merge factors (rank 0)
-  float part_m[QG], part_l[QG];
-  float part_o[QG][128];
+  // rank 0 only: the partial results (m, l, o) of every CTA of the cluster,
+  // written by each CTA into rank 0's copy before the cluster barrier
+  float cm[16][QG], cl[16][QG];
+  alignas(16) float co[16][QG][128];
   uint64_t full[MQ_NS], empty[MQ_NS];
 };
 
@@ -569,7 +580,8 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   __syncthreads();
   pdl_wait();  // the queries and the cache come from earlier kernels
   pdl_trigger();
-  // the query words first: issued after the tile copies they would queue behind them
+  // the query words and the 4-bit list first: issued after the tile copies
+  // they would queue behind them
   const int qcol = QG == 4 ? (g >> 1) : g;  // query of this lane's column of the score MMA
   uint32_t qw[16];  // dims 32 t4 .. 32 t4 + 31 as bf16 pairs
 #pragma unroll
@@ -590,10 +602,12 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     tma_load_2d(&sm.ksc[st][0][0], &tmKs, &sm.full[st], h4, t0);
     tma_load_2d(&sm.vsc[st][0][0], &tmVs, &sm.full[st], h4, t0);
   };
-  int n_issued = 0;
-  if (tid == 0)
-    for (; n_issued < min(MQ_NS, n_tiles); ++n_issued) issue(n_issued);
   for (int i = tid; i < n4; i += MQ_TT) sm.s_keep[i] = __ldg(p.keep4 + i);
+  // tile 0 alone first: with every CTA's second tile in flight too, the
+  // first ones would land only with the whole cache; tile 1 is issued once
+  // tile 0 is in, and streams while it is computed
+  int n_issued = 0;
+  if (tid == 0 && n_tiles > 0) issue(n_issued++);
 
   // the query operand of the score MMA: pair pi of chunk t4, bf16 q_a / 16 | q_(a+4)
   uint32_t qb[16];
@@ -640,6 +654,7 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   for (; k < n_tiles; ++k) {
     const int st = k % MQ_NS, t0 = t_begin + k * MQ_TT;
     if (!mbar_wait(&sm.full[st], (k / MQ_NS) & 1, p.timeout_ns, nullptr)) { ok = false; break; }
+    if (tid == 0 && k == 0 && n_issued < n_tiles) issue(n_issued++);  // into the stage not used yet
     const int tw0 = t0 + 32 * warp;
     uint32_t m4 = 0u;  // bit i: token tw0 + i is kept at 4 bits
     if (k4lo < k4hi) {
@@ -848,7 +863,10 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       sm.wl[warp][qi] = l_run[q];
     }
   __syncthreads();
-  if (tid < QG) {  // the warps' factors 2^(m_w - M) and the CTA's (M, L)
+  // the warps' factors 2^(m_w - M), and this CTA's (M, L, O) written into
+  // rank 0's slots (distributed shared memory stores, ordered by the
+  // release / acquire of the cluster barrier)
+  if (tid < QG) {
     float M = -INFINITY;
 #pragma unroll
     for (int ww = 0; ww < MQ_WARPS; ++ww) M = fmaxf(M, sm.wm[ww][tid]);
@@ -859,55 +877,45 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
       sm.wf[ww][tid] = f;
       L = fmaf(f, sm.wl[ww][tid], L);
     }
-    sm.part_m[tid] = M;
-    sm.part_l[tid] = L;
+    st_dsmem_f32(map_shared_rank(smem_u32(&sm.cm[rank][tid]), 0u), M);
+    st_dsmem_f32(map_shared_rank(smem_u32(&sm.cl[rank][tid]), 0u), L);
   }
   __syncthreads();
-  for (int i = tid; i < QG * D; i += MQ_TT) {
-    const int q = i / D, d = i - q * D;
-    float O = 0.f;
+  for (int i = tid; i < QG * D / 4; i += MQ_TT) {  // 4 dimensions an item
+    const int q = i / (D / 4), d = 4 * (i - q * (D / 4));
+    float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-    for (int ww = 0; ww < MQ_WARPS; ++ww) O = fmaf(sm.wf[ww][q], sm.u.wo[ww][q][d], O);
-    sm.part_o[q][d] = O;
+    for (int ww = 0; ww < MQ_WARPS; ++ww) {
+      const float f = sm.wf[ww][q];
+      const float4 x = *reinterpret_cast<const float4*>(&sm.u.wo[ww][q][d]);
+      O.x = fmaf(f, x.x, O.x); O.y = fmaf(f, x.y, O.y); O.z = fmaf(f, x.z, O.z); O.w = fmaf(f, x.w, O.w);
+    }
+    st_dsmem_v4f32(map_shared_rank(smem_u32(&sm.co[rank][q][d]), 0u), O);
   }
   cluster_sync();
+  // rank 0 merges the S partial results from its own shared memory; the
+  // other CTAs are done (nothing reads their shared memory any more)
   if (rank == 0 && !bad) {  // block-uniform
     if (tid < nb) {  // the ranks' factors 2^(m_r - M) / L
-      float mr[16], lr[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        mr[r] = -INFINITY; lr[r] = 0.f;
-        if (r < S) {
-          mr[r] = ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_m[tid]), static_cast<uint32_t>(r)));
-          lr[r] = ld_dsmem_f32(map_shared_rank(smem_u32(&sm.part_l[tid]), static_cast<uint32_t>(r)));
-        }
-      }
       float M = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < 16; ++r) M = fmaxf(M, mr[r]);
+      for (int r = 0; r < S; ++r) M = fmaxf(M, sm.cm[r][tid]);
       float L = 0.f;
-#pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        mr[r] = mr[r] == -INFINITY ? 0.f : exp2f(mr[r] - M);
-        L = fmaf(mr[r], lr[r], L);
+      for (int r = 0; r < S; ++r) {
+        const float f = sm.cm[r][tid] == -INFINITY ? 0.f : exp2f(sm.cm[r][tid] - M);
+        sm.rf[tid][r] = f;
+        L = fmaf(f, sm.cl[r][tid], L);
       }
-#pragma unroll
-      for (int r = 0; r < 16; ++r) sm.rf[tid][r] = mr[r] / L;
+      const float inv = 1.f / L;
+      for (int r = 0; r < S; ++r) sm.rf[tid][r] *= inv;
     }
     __syncthreads();
     for (int i = tid; i < nb * D; i += MQ_TT) {
       const int q = i / D, d = i - q * D;
-      const uint32_t oa = smem_u32(&sm.part_o[q][d]);
-      float orr[16];
-#pragma unroll
-      for (int r = 0; r < 16; ++r) orr[r] = r < S ? ld_dsmem_f32(map_shared_rank(oa, static_cast<uint32_t>(r))) : 0.f;
       float o = 0.f;
-#pragma unroll
-      for (int r = 0; r < 16; ++r) o = fmaf(sm.rf[q][r], orr[r], o);
+      for (int r = 0; r < S; ++r) o = fmaf(sm.rf[q][r], sm.co[r][q][d], o);
       p.out[(static_cast<int64_t>(b0 + q) * p.H + h) * D + d] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
     }
   }
-  cluster_sync();  // peers keep their shared memory until rank 0 is done
 }
 }  // namespace attn
 
