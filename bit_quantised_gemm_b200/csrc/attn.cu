@@ -13,7 +13,7 @@
 // through distributed shared memory by cluster rank 0, so no global scratch
 // is needed. The rows of one head are 3D/8 bytes every H * 3D/8 bytes in the
 // cache, so each tile's K rows, V rows and their scales arrive by TMA (2-D
-// boxes, one row per token) into a two-stage ring: the next tile is in
+// boxes, one row per token) into a ring of stages: the next tiles are in
 // flight while the current one is computed.
 //
 // D = 128 (`kv_attention_mma_kernel`, below): both products on the warp-level
@@ -402,9 +402,9 @@ kv_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 // ---------------------------------------------------------------------------
 // D = 128, up to QG queries per (head, query group): both products on the
 // warp-level bf16 tensor-core MMA (m16n8k16, fp32 accumulation). A CTA of 8
-// warps walks its token range in 256-token tiles staged by TMA (as above, a
-// two-stage ring); warp w owns tokens [32 w, 32 w + 32) of every tile, in two
-// steps of 16.
+// warps walks its token range in 256-token tiles staged by TMA (a
+// three-stage ring, one CTA an SM); warp w owns tokens [32 w, 32 w + 32) of
+// every tile, in two steps of 16.
 //
 // Scores, S[t][n] = sum_k K[t][k] Q[k][n]: A = 16 tokens x 16 dims of
 // 3-bit codes, B = 16 dims x 8 query columns. The order of the dimensions
@@ -446,7 +446,7 @@ kv_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 // per query.
 constexpr int MQ_WARPS = 8;
 constexpr int MQ_TT = 32 * MQ_WARPS;  // tokens per tile = threads per CTA
-constexpr int MQ_NS = 2;
+constexpr int MQ_NS = 3;
 
 template <int QG>
 struct SmemMQ {
@@ -531,7 +531,7 @@ __device__ __forceinline__ uint32_t v_operand(const uint32_t (&wa)[4], const uin
 }
 
 template <int QG>
-constexpr int mq_ctas_per_sm() { return QG == 4 ? 2 : 1; }
+constexpr int mq_ctas_per_sm() { return 1; }  // shared memory: one CTA an SM
 
 __device__ __forceinline__ int lower_bound_i32(const int32_t* a, int lo, int hi, int key) {
   while (lo < hi) {
@@ -603,9 +603,9 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
     tma_load_2d(&sm.vsc[st][0][0], &tmVs, &sm.full[st], h4, t0);
   };
   for (int i = tid; i < n4; i += MQ_TT) sm.s_keep[i] = __ldg(p.keep4 + i);
-  // tile 0 alone first: with every CTA's second tile in flight too, the
-  // first ones would land only with the whole cache; tile 1 is issued once
-  // tile 0 is in, and streams while it is computed
+  // tile 0 alone first: with every CTA's later tiles in flight too, the
+  // first ones would land only with the whole cache; the next MQ_NS - 1 are
+  // issued once tile 0 is in, and stream while it is computed
   int n_issued = 0;
   if (tid == 0 && n_tiles > 0) issue(n_issued++);
 
@@ -654,7 +654,8 @@ kv_attention_mma_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_co
   for (; k < n_tiles; ++k) {
     const int st = k % MQ_NS, t0 = t_begin + k * MQ_TT;
     if (!mbar_wait(&sm.full[st], (k / MQ_NS) & 1, p.timeout_ns, nullptr)) { ok = false; break; }
-    if (tid == 0 && k == 0 && n_issued < n_tiles) issue(n_issued++);  // into the stage not used yet
+    if (tid == 0 && k == 0)  // into the stages not used yet
+      while (n_issued < min(MQ_NS, n_tiles)) issue(n_issued++);
     const int tw0 = t0 + 32 * warp;
     uint32_t m4 = 0u;  // bit i: token tw0 + i is kept at 4 bits
     if (k4lo < k4hi) {
