@@ -421,7 +421,8 @@ int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_
   if (!q || !k_codes3 || !k_scale || !v_codes3 || !v_scale || !out)
     return fail(BITLINEAR_ERR_INVALID_ARG, "kv_attention_3bit: null pointer");
   if (!aligned16(q) || !aligned16(k_codes3) || !aligned16(v_codes3) || !aligned16(k_scale) ||
-      !aligned16(v_scale) || !aligned16(out))
+      !aligned16(v_scale) || !aligned16(out) ||
+      (n_keep4 > 0 && (!aligned16(k_codes4) || !aligned16(v_codes4))))
     return fail(BITLINEAR_ERR_ALIGNMENT, "kv_attention_3bit: q, codes, scales and out must be 16-byte aligned");
   const char* why = nullptr;
   cudaError_t e = blt::launch_kv_attention(q, B, H, D, T, k_codes3, k_codes4, k_scale, v_codes3,

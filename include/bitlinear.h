@@ -248,8 +248,8 @@ int kv_keep4_positions(const int32_t* token_ids, int64_t T, const int32_t* speci
  *   keep4_pos  device int32 [n_keep4], strictly increasing, n_keep4 <= 1024
  *   out        device bf16 [B x H x D]
  *   dev_status as for the GEMMs (bounded waits on the cache tiles)
- * Requires D in {128, 256}, H % 4 == 0, T >= 1, every pointer but codes4 and
- * keep4_pos 16-byte aligned; B == 0 launches nothing.
+ * Requires D in {128, 256}, H % 4 == 0, T >= 1, every pointer but keep4_pos
+ * 16-byte aligned (codes4 only when n_keep4 > 0); B == 0 launches nothing.
  */
 int kv_attention_3bit(const uint16_t* q, int64_t B, int64_t H, int64_t D, int64_t T,
                       const uint8_t* k_codes3, const uint8_t* k_codes4, const float* k_scale,

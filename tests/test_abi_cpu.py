@@ -123,6 +123,8 @@ def test_kv_attention_argument_errors():
     assert call(n4=65, keep=FAKE, k4=FAKE, v4=FAKE) == _lib.ERR_INVALID_ARG  # more than T
     assert call(q=None) == _lib.ERR_INVALID_ARG
     assert call(out=FAKE + 2) == _lib.ERR_ALIGNMENT
+    assert call(n4=1, keep=FAKE, k4=FAKE + 8, v4=FAKE) == _lib.ERR_ALIGNMENT  # 4-bit rows: 16-byte aligned
+    assert call(n4=1, keep=FAKE, k4=FAKE, v4=FAKE + 4) == _lib.ERR_ALIGNMENT
     assert call(B=0) == _lib.OK
 
 
