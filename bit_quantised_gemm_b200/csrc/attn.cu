@@ -441,9 +441,10 @@ kv_attention_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_consta
 // step: every lane forms the partial score over its 16 dimensions, the
 // lanes sum them, and each lane adds its 16 dimensions of the value row.
 // Their rows are prefetched into L2 when the kernel starts. The 8 warps then
-// merge through shared memory and the CTAs of the cluster through
-// distributed shared memory, each with its factors 2^(m - M) computed once
-// per query.
+// merge through shared memory; every CTA stores its partial result (m, l, o)
+// into rank 0's shared memory (distributed shared-memory stores ordered by
+// the cluster barrier), and rank 0 merges them. Both merges take their
+// factors 2^(m - M) once per query.
 constexpr int MQ_WARPS = 8;
 constexpr int MQ_TT = 32 * MQ_WARPS;  // tokens per tile = threads per CTA
 constexpr int MQ_NS = 3;
