@@ -81,7 +81,7 @@ struct Layout {
   static constexpr int OFF_WP = OFF_B + S_B * B_BYTES;
   static constexpr int OFF_STG = OFF_WP + S_W * WP_BYTES;  // epilogue staging, 4 KB per warp
   static constexpr int OFF_BAR = OFF_STG + 4 * 4096;
-  static constexpr int N_BARS = 2 * S_TMA + 2 * S_W + 2 * S_B + 2 * 2 + 1;
+  static constexpr int N_BARS = 2 * S_TMA + 2 * S_W + 2 * S_B + 2 * 2 + 2;
   static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + slack for 1024-byte alignment
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -114,6 +114,106 @@ __device__ __forceinline__ int kb_at(int kb, int rot, int num_kb) {
   return k >= num_kb ? k - num_kb : k;
 }
 
+// Every group's weight scale and the group ends, in registers.
+struct EpiScales {
+  float gam[8];
+  int ge[7];  // past the last group: none
+  __device__ __forceinline__ void load(const Params& p) {
+#pragma unroll
+    for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
+#pragma unroll
+    for (int g = 0; g < 7; ++g) ge[g] = g < p.G - 1 ? p.group_end[g] : 0x7FFFFFFF;
+  }
+};
+
+// One 64-column chunk of a tile's accumulator (TMEM columns col .. col + 63,
+// lane quadrant q) -> bf16 y[m0 + q * 32 .. + 31][n .. n + 63], staged in the
+// 4 KB shared-memory block stg (or the raw accumulators straight to global).
+template <bool FP4>
+__device__ __forceinline__ void epi_chunk(const Params& p, const CUtensorMap* tmY, uint32_t tmem_base, int lane,
+                                          const EpiScales& es, int m0, int n, uint32_t col, int q, uint32_t stg,
+                                          float xs_m, bool row_ok, int m) {
+    auto grp = [&](int cc) {
+      int g = 0;
+#pragma unroll
+      for (int i = 0; i < 7; ++i) g += cc >= es.ge[i] ? 1 : 0;
+      return g;
+    };
+        uint32_t r[64];
+        tmem_ld64(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
+        tmem_ld_wait();
+        if (p.out_mode == kOutBf16) {
+          // y = acc * (xs[m] * gamma[group(n)]); one scale per 64-column chunk
+          // unless the chunk straddles a group boundary
+          const int g0 = grp(n);
+          const int g1 = grp(min(n + 63, p.N - 1));
+          float s0 = 0.f;
+#pragma unroll
+          for (int g = 0; g < 8; ++g) s0 = (g == g0) ? es.gam[g] : s0;
+          s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
+            // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
+            // (1.5 * 2^23 + acc) - 1.5 * 2^23
+            const float f = FP4 ? __uint_as_float(r[i])
+                                : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
+            r[i] = __float_as_uint(f);
+          }
+          if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
+#pragma unroll
+            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), s0));
+          } else {
+            // the chunk crosses group boundaries: one pass per group touched
+            // (a dynamic loop, so the common path above is not predicated)
+#pragma unroll 1
+            for (int g = g0; g <= g1; ++g) {
+              int lo = 0, hi = 0x7FFFFFFF;
+#pragma unroll
+              for (int j = 0; j < 7; ++j) {
+                lo = (j == g - 1) ? es.ge[j] : lo;
+                hi = (j == g) ? es.ge[j] : hi;
+              }
+              float t = 0.f;
+#pragma unroll
+              for (int j = 0; j < 8; ++j) t = (j == g) ? es.gam[j] : t;
+              const float sg = __fmul_rn(xs_m, t);
+#pragma unroll
+              for (int i = 0; i < 64; ++i)
+                r[i] = (n + i >= lo && n + i < hi) ? __float_as_uint(__fmul_rn(__uint_as_float(r[i]), sg))
+                                                   : r[i];
+            }
+          }
+          // stage the warp's 32 x 64 bf16 block (128 B per row, 16-byte unit v
+          // of row r at v ^ (r & 7): the 128-byte swizzle of the output tensor
+          // map) and write it with one TMA store; rows past M and columns
+          // past N are clipped by the map
+          if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
+          __syncwarp();
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                         pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(tmY, stg, n, m0 + q * 32);
+            bulk_commit();
+          }
+        } else if (row_ok) {
+          uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            if (n + 4 * v >= p.N) break;
+            reinterpret_cast<uint4*>(orow)[v] =
+                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+          }
+        }
+}
+
 template <bool FP4, bool PAIR, bool MX>
 __global__ void __launch_bounds__(THREADS, 1)
 bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -144,6 +244,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   uint64_t* tfull = bempty + S_B;           // accumulator ready (both CTAs)
   uint64_t* tempty = tfull + 2;             // accumulator drained (even CTA: both epilogues)
   uint64_t* mma_done = tempty + 2;          // all MMAs retired (teardown)
+  uint64_t* last_acc = mma_done + 1;        // the epilogue warps have this CTA's last accumulator (used once)
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + L::OFF_MISC);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + L::OFF_MISC + 4);
 
@@ -160,6 +261,7 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     for (int i = 0; i < S_B; ++i) { mbar_init(&bfull[i], PAIR ? 2 * UW : UW); mbar_init(&bempty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&tfull[i], 1); mbar_init(&tempty[i], PAIR ? 8 : 4); }
     mbar_init(mma_done, 1);
+    mbar_init(last_acc, 4);
     *s_abort = 0;
     fence_mbar_init();
     prefetch_tensormap(&tmA);
@@ -206,6 +308,10 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     *s_abort = 1;
     report_status(p.status, BITLINEAR_STATUS_TIMEOUT);
   };
+  // the last tile's epilogue chunks are spread over the warp sets: chunk c
+  // by the epilogue warps (c = 0), the unpack warps 8-11 (1) and 12-15 (2),
+  // the producer / issuer warps 0-3 (3), each set on all four lane quadrants
+  constexpr int NCH = BN / 64;
   // global bytes per activation box (the padded f8f6f4 form reads half of what it stages)
   constexpr uint32_t A_TX = (FP4 && !MX) ? L::A_BYTES / 2 : L::A_BYTES;
 
@@ -324,18 +430,8 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int q = warp & 3;  // TMEM lane quadrant
     const uint32_t tempty_addr0 = lead(&tempty[0]);
     const uint32_t stg = smem_u32(smem + L::OFF_STG) + q * 4096;  // this warp's staging block
-    float gam[8];  // every group's weight scale, loaded once
-#pragma unroll
-    for (int g = 0; g < 8; ++g) gam[g] = (p.out_mode == kOutBf16 && g < p.G) ? __ldg(p.gamma + g) : 0.f;
-    int ge[7];     // group ends in registers (past the last group: none)
-#pragma unroll
-    for (int g = 0; g < 7; ++g) ge[g] = g < p.G - 1 ? p.group_end[g] : 0x7FFFFFFF;
-    auto grp = [&](int col) {
-      int g = 0;
-#pragma unroll
-      for (int i = 0; i < 7; ++i) g += col >= ge[i] ? 1 : 0;
-      return g;
-    };
+    EpiScales es;
+    es.load(p);
     pdl_wait();  // row scales come from the previous kernel; y may still be read by it
     uint32_t tl = 0;
     for (int tile = cta_slot; tile < p.num_tiles; tile += cta_stride, ++tl) {
@@ -348,83 +444,17 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const float xs_m = (row_ok && p.out_mode == kOutBf16) ? __ldg(p.xs + m) : 0.f;
       if (!mbar_wait(&tfull[acc], aph, tmo, s_abort)) { fail(); break; }
       tc_fence_after();
+      // the last tile's chunks are shared with the other warps (below): this
+      // warp set writes chunk 0 of it, and tells them the accumulator is ready
+      // (a barrier of its own: a wait on tfull by parity alone cannot tell the
+      // last tile's phase from an earlier one)
+      const bool last = tile + cta_stride >= p.num_tiles;
+      if (last && lane == 0) mbar_arrive(last_acc);
 #pragma unroll 1
-      for (int c = 0; c < BN / 64; ++c) {
+      for (int c = 0; c < (last ? 1 : NCH); ++c) {
         const int n = n0 + c * 64;
         if (n >= p.N) break;  // warp-uniform
-        uint32_t r[64];
-        tmem_ld64(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + acc * BN + c * 64, r);
-        tmem_ld_wait();
-        if (p.out_mode == kOutBf16) {
-          // y = acc * (xs[m] * gamma[group(n)]); one scale per 64-column chunk
-          // unless the chunk straddles a group boundary
-          const int g0 = grp(n);
-          const int g1 = grp(min(n + 63, p.N - 1));
-          float s0 = 0.f;
-#pragma unroll
-          for (int g = 0; g < 8; ++g) s0 = (g == g0) ? gam[g] : s0;
-          s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
-#pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
-            // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
-            // (1.5 * 2^23 + acc) - 1.5 * 2^23
-            const float f = FP4 ? __uint_as_float(r[i])
-                                : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
-            r[i] = __float_as_uint(f);
-          }
-          if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
-#pragma unroll
-            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), s0));
-          } else {
-            // the chunk crosses group boundaries: one pass per group touched
-            // (a dynamic loop, so the common path above is not predicated)
-#pragma unroll 1
-            for (int g = g0; g <= g1; ++g) {
-              int lo = 0, hi = 0x7FFFFFFF;
-#pragma unroll
-              for (int j = 0; j < 7; ++j) {
-                lo = (j == g - 1) ? ge[j] : lo;
-                hi = (j == g) ? ge[j] : hi;
-              }
-              float t = 0.f;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) t = (j == g) ? gam[j] : t;
-              const float sg = __fmul_rn(xs_m, t);
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                r[i] = (n + i >= lo && n + i < hi) ? __float_as_uint(__fmul_rn(__uint_as_float(r[i]), sg))
-                                                   : r[i];
-            }
-          }
-          // stage the warp's 32 x 64 bf16 block (128 B per row, 16-byte unit v
-          // of row r at v ^ (r & 7): the 128-byte swizzle of the output tensor
-          // map) and write it with one TMA store; rows past M and columns
-          // past N are clipped by the map
-          if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
-          __syncwarp();
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&tmY, stg, n, m0 + q * 32);
-            bulk_commit();
-          }
-        } else if (row_ok) {
-          uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
-#pragma unroll
-          for (int v = 0; v < 16; ++v) {
-            if (n + 4 * v >= p.N) break;
-            reinterpret_cast<uint4*>(orow)[v] =
-                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-          }
-        }
+        epi_chunk<FP4>(p, &tmY, tmem_base, lane, es, m0, n, acc * BN + c * 64, q, stg, xs_m, row_ok, m);
       }
       tc_fence_before();
       __syncwarp();
@@ -502,6 +532,37 @@ bitlinear_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (PAIR) mbar_arrive_cluster(bfull_addr0 + 8u * b);
           else      mbar_arrive(&bfull[b]);
         }
+      }
+    }
+  }
+
+  // ---- the last tile's other chunks: warp set k (1: warps 8-11, 2: 12-15,
+  // 3: 0-3) writes chunk k of this CTA's last tile once its accumulator is
+  // ready, staging in the unpacked-weight ring (no MMA reads it any more)
+  {
+    __syncwarp();
+    const int set = warp >= 8 ? 1 + ((warp - 8) >> 2) : (warp < 4 ? 3 : 0);
+    const int count = cta_slot < p.num_tiles ? (p.num_tiles - 1 - cta_slot) / cta_stride + 1 : 0;
+    if (set > 0 && set < NCH && count > 0 && !*s_abort) {
+      const int q = warp & 3;
+      const uint32_t tl = static_cast<uint32_t>(count - 1);
+      const int tile = cta_slot + static_cast<int>(tl) * cta_stride;
+      const int m0 = (tile % p.tiles_m) * TILE_M + static_cast<int>(rank) * BM;
+      const int n = (tile / p.tiles_m) * BN + set * 64;
+      const uint32_t acc = tl & 1;
+      const int m = m0 + q * 32 + lane;
+      const bool row_ok = m < p.M;
+      EpiScales es;
+      es.load(p);
+      pdl_wait();  // as for the epilogue warps
+      const float xs_m = (row_ok && p.out_mode == kOutBf16) ? __ldg(p.xs + m) : 0.f;
+      if (!mbar_wait(last_acc, 0, tmo, s_abort)) {
+        fail();
+      } else if (n < p.N) {
+        tc_fence_after();
+        epi_chunk<FP4>(p, &tmY, tmem_base, lane, es, m0, n, acc * BN + set * 64, q, sB + ((set - 1) * 4 + q) * 4096,
+                       xs_m, row_ok, m);
+        if (lane == 0) bulk_wait_all();  // its output stores complete before the CTA exits
       }
     }
   }
