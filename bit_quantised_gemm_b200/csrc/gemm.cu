@@ -133,85 +133,85 @@ template <bool FP4>
 __device__ __forceinline__ void epi_chunk(const Params& p, const CUtensorMap* tmY, uint32_t tmem_base, int lane,
                                           const EpiScales& es, int m0, int n, uint32_t col, int q, uint32_t stg,
                                           float xs_m, bool row_ok, int m) {
-    auto grp = [&](int cc) {
-      int g = 0;
+  auto grp = [&](int cc) {
+    int g = 0;
 #pragma unroll
-      for (int i = 0; i < 7; ++i) g += cc >= es.ge[i] ? 1 : 0;
-      return g;
-    };
-        uint32_t r[64];
-        tmem_ld64(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
-        tmem_ld_wait();
-        if (p.out_mode == kOutBf16) {
-          // y = acc * (xs[m] * gamma[group(n)]); one scale per 64-column chunk
-          // unless the chunk straddles a group boundary
-          const int g0 = grp(n);
-          const int g1 = grp(min(n + 63, p.N - 1));
-          float s0 = 0.f;
+    for (int i = 0; i < 7; ++i) g += cc >= es.ge[i] ? 1 : 0;
+    return g;
+  };
+  uint32_t r[64];
+  tmem_ld64(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + col, r);
+  tmem_ld_wait();
+  if (p.out_mode == kOutBf16) {
+    // y = acc * (xs[m] * gamma[group(n)]); one scale per 64-column chunk
+    // unless the chunk straddles a group boundary
+    const int g0 = grp(n);
+    const int g1 = grp(min(n + 63, p.N - 1));
+    float s0 = 0.f;
 #pragma unroll
-          for (int g = 0; g < 8; ++g) s0 = (g == g0) ? es.gam[g] : s0;
-          s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
+    for (int g = 0; g < 8; ++g) s0 = (g == g0) ? es.gam[g] : s0;
+    s0 = __fmul_rn(xs_m, s0);  // y = acc * (xs[m] * gamma[group(n)])
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
-            // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
-            // (1.5 * 2^23 + acc) - 1.5 * 2^23
-            const float f = FP4 ? __uint_as_float(r[i])
-                                : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
-            r[i] = __float_as_uint(f);
-          }
-          if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
+    for (int i = 0; i < 64; ++i) {
+      // FP4: the fp32 accumulator. int8: exact int32 -> fp32 for
+      // |acc| < 2^22 (|acc| <= 128 K) on the integer/FMA pipes:
+      // (1.5 * 2^23 + acc) - 1.5 * 2^23
+      const float f = FP4 ? __uint_as_float(r[i])
+                          : __fsub_rn(__int_as_float(static_cast<int32_t>(r[i]) + 0x4B400000), 12582912.f);
+      r[i] = __float_as_uint(f);
+    }
+    if (g0 == g1) {  // warp-uniform: the whole chunk in one scale group
 #pragma unroll
-            for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), s0));
-          } else {
-            // the chunk crosses group boundaries: one pass per group touched
-            // (a dynamic loop, so the common path above is not predicated)
+      for (int i = 0; i < 64; ++i) r[i] = __float_as_uint(__fmul_rn(__uint_as_float(r[i]), s0));
+    } else {
+      // the chunk crosses group boundaries: one pass per group touched
+      // (a dynamic loop, so the common path above is not predicated)
 #pragma unroll 1
-            for (int g = g0; g <= g1; ++g) {
-              int lo = 0, hi = 0x7FFFFFFF;
+      for (int g = g0; g <= g1; ++g) {
+        int lo = 0, hi = 0x7FFFFFFF;
 #pragma unroll
-              for (int j = 0; j < 7; ++j) {
-                lo = (j == g - 1) ? es.ge[j] : lo;
-                hi = (j == g) ? es.ge[j] : hi;
-              }
-              float t = 0.f;
-#pragma unroll
-              for (int j = 0; j < 8; ++j) t = (j == g) ? es.gam[j] : t;
-              const float sg = __fmul_rn(xs_m, t);
-#pragma unroll
-              for (int i = 0; i < 64; ++i)
-                r[i] = (n + i >= lo && n + i < hi) ? __float_as_uint(__fmul_rn(__uint_as_float(r[i]), sg))
-                                                   : r[i];
-            }
-          }
-          // stage the warp's 32 x 64 bf16 block (128 B per row, 16-byte unit v
-          // of row r at v ^ (r & 7): the 128-byte swizzle of the output tensor
-          // map) and write it with one TMA store; rows past M and columns
-          // past N are clipped by the map
-          if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
-          __syncwarp();
-#pragma unroll
-          for (int v = 0; v < 8; ++v)
-            st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
-                         pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(tmY, stg, n, m0 + q * 32);
-            bulk_commit();
-          }
-        } else if (row_ok) {
-          uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
-#pragma unroll
-          for (int v = 0; v < 16; ++v) {
-            if (n + 4 * v >= p.N) break;
-            reinterpret_cast<uint4*>(orow)[v] =
-                make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
-          }
+        for (int j = 0; j < 7; ++j) {
+          lo = (j == g - 1) ? es.ge[j] : lo;
+          hi = (j == g) ? es.ge[j] : hi;
         }
+        float t = 0.f;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) t = (j == g) ? es.gam[j] : t;
+        const float sg = __fmul_rn(xs_m, t);
+#pragma unroll
+        for (int i = 0; i < 64; ++i)
+          r[i] = (n + i >= lo && n + i < hi) ? __float_as_uint(__fmul_rn(__uint_as_float(r[i]), sg))
+                                             : r[i];
+      }
+    }
+    // stage the warp's 32 x 64 bf16 block (128 B per row, 16-byte unit v
+    // of row r at v ^ (r & 7): the 128-byte swizzle of the output tensor
+    // map) and write it with one TMA store; rows past M and columns
+    // past N are clipped by the map
+    if (lane == 0) bulk_wait_read_all();  // the previous block has left the buffer
+    __syncwarp();
+#pragma unroll
+    for (int v = 0; v < 8; ++v)
+      st_shared_v4(stg + lane * 128 + ((v ^ (lane & 7)) << 4),
+                   pack_bf16x2(__uint_as_float(r[8 * v + 0]), __uint_as_float(r[8 * v + 1])),
+                   pack_bf16x2(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                   pack_bf16x2(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                   pack_bf16x2(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      tma_store_2d(tmY, stg, n, m0 + q * 32);
+      bulk_commit();
+    }
+  } else if (row_ok) {
+    uint32_t* orow = reinterpret_cast<uint32_t*>(p.out) + static_cast<int64_t>(m) * p.ldo + n;
+#pragma unroll
+    for (int v = 0; v < 16; ++v) {
+      if (n + 4 * v >= p.N) break;
+      reinterpret_cast<uint4*>(orow)[v] =
+          make_uint4(r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+    }
+  }
 }
 
 template <bool FP4, bool PAIR, bool MX>
